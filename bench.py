@@ -1,0 +1,456 @@
+"""Benchmark: one decode step of paged KV-cache attention on B200, per the benchmark contract.
+
+A step is one pass of the whole hot path over one batch: copy-on-write block copies (when
+the workload has any), the cache update of one new token per sequence, and the decode
+attention.  Inputs are seeded synthetic tensors resident in HBM.  The JSON line reports
+
+* ``value``: algorithmic bytes of the step / step time (GB/s), summed over ranks;
+* ``tokens_per_s``: decode tokens (one per sequence) per second, summed over ranks;
+* ``roofline``: the decode kernel alone, timed with CUDA events on its stream, against the
+  measured HBM copy bandwidth;
+* ``e2e``: the same metric through the public API with the step's inputs copied from pinned
+  host memory and the output copied back, inside the timed region;
+* ``cpu_baseline``: the fp64 oracle on this host's cores on a bounded sample (rank 0, N=1).
+
+``--impl reference`` times the oracle (the CPU reference of this method) instead.
+Multi-GPU (torchrun): every rank runs its own replica (weak scaling, no data-path
+collective); ranks only agree on the barrier and on the max step time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_344_b200 import workloads  # noqa: E402
+
+METRIC = "paged decode attention: achieved HBM GB/s (% of B200 peak) and decode tokens/s"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+DESCR = {
+    "tiny": "tiny fp32: B=4, lengths {1,7,16,33}+1, Hq=Hkv=4, D=64, bs=16, pool 32",
+    "mha": "MHA bf16: B=64, Hq=Hkv=40, D=128, bs=16, seq_len U[128,2048]+1, pool 1.25x, shuffled",
+    "gqa16": "GQA bf16: B=256, Hq=32, Hkv=8, D=128, bs=16, lognormal(1024,0.8) in [16,4096]+1",
+    "gqa32": "GQA bf16: B=256, Hq=32, Hkv=8, D=128, bs=32, lognormal(1024,0.8) in [16,4096]+1",
+    "long": "long-context GQA bf16: B=8, Hq=64, Hkv=8, D=128, bs=16, seq_len U[32768,131072]+1",
+    "share_fork": "shared-prefix bf16: 32 groups x 4 branches, Hq=32, Hkv=8, D=128, bs=16, "
+                  "prefix 1024+U[1,15] shared (refcount 4), CoW of the partial block",
+    "share_tails": "shared-prefix bf16: 32 groups x 4 branches, Hq=32, Hkv=8, D=128, bs=16, "
+                   "1024-token shared prefix + private tails U[0,256]",
+}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_344_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", f"decode_{config}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    if not m or not s or s.group(1) != kernel_source_sha():
+        return None
+    return float(m.group(1))
+
+
+# ----------------------------------------------------------------------------------------
+# clocks during the timed region (NVML, sampled in a thread)
+# ----------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz, self.ok = [], 0, None, False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report clocks as unavailable
+            self.err = str(e)
+
+    def _handle(self, idx):
+        import torch
+        nv = self.nv
+        try:
+            p = torch.cuda.get_device_properties(idx)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId_v2(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(idx)
+
+    def _reasons(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return f(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons())
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+    def rejected(self):
+        s = self.summary()
+        bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+        if bad & set(s["reasons"]):
+            return True
+        return bool(s["sm_mhz"] and s["sm_max_mhz"] and s["sm_mhz"] < 0.5 * s["sm_max_mhz"]
+                    and not s["reasons"])
+
+
+# ----------------------------------------------------------------------------------------
+# CPU side: the oracle on a bounded sample
+# ----------------------------------------------------------------------------------------
+def oracle_sample(wl, host_pool, budget_rows: int):
+    """Sequences 0..n-1 whose rows stay under ``budget_rows`` row-tokens; returns the oracle
+    inputs for them and their algorithmic bytes."""
+    lens = wl.seq_lens_post
+    acc, n = 0, 0
+    for b in range(wl.B):
+        acc += int(lens[b]) * wl.Hq
+        n = b + 1
+        if acc >= budget_rows:
+            break
+    return n
+
+
+def time_oracle(wl, host, n_seq: int):
+    import oracle
+    q = np.ascontiguousarray(host["q"][:n_seq])
+    bt = np.ascontiguousarray(wl.block_tables[:n_seq])
+    sl = np.ascontiguousarray(wl.seq_lens_post[:n_seq])
+    t0 = time.perf_counter()
+    oracle.paged_decode(q, host["k_cache"], host["v_cache"], bt, sl, wl.scale)
+    dt = time.perf_counter() - t0
+    blocks = sum(-(-int(L) // wl.bs) for L in sl)
+    nbytes = blocks * wl.block_bytes * 2 + 2 * n_seq * wl.Hq * wl.D * wl.elt + blocks * 4
+    return dt, nbytes, int(sl.sum()), oracle.num_threads()
+
+
+def host_pool_from(dev, wl):
+    import torch
+    out = {}
+    for k in ("q", "k_cache", "v_cache"):
+        t = dev[k].detach().cpu().contiguous()
+        out[k] = t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+    return out
+
+
+# ----------------------------------------------------------------------------------------
+# GPU side
+# ----------------------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import paged_kv_cache_344_b200 as pkv
+
+    torch.cuda.set_device(local_rank)
+    dev_name = f"cuda:{local_rank}"
+    wl = workloads.make(args.config)
+    dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
+    meta = {
+        "block_tables": torch.from_numpy(wl.block_tables).to(dev_name),
+        "seq_lens": torch.from_numpy(wl.seq_lens_post).to(dev_name),
+        "slot_mapping": torch.from_numpy(wl.slot_mapping).to(dev_name),
+        "cow_pairs": torch.from_numpy(wl.cow_pairs).to(dev_name),
+    }
+    ws_bytes = pkv.paged_attention_decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D,
+                                                         wl.max_seq_len, wl.bs, 0)
+    ws = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev_name)
+    out = torch.empty_like(dev["q"])
+    has_cow = len(wl.cow_pairs) > 0
+    launches_per_step = 2 + int(has_cow)
+    stream = torch.cuda.current_stream()
+
+    # The CoW step restores its own precondition: copying block src -> dst again is
+    # idempotent, and rewriting the same token to the same slot is too.
+    def step(d_in, ev_pair=None):
+        if has_cow:
+            pkv.copy_blocks(d_in["k_cache"], d_in["v_cache"], d_in["cow_pairs"])
+        pkv.paged_kv_write(d_in["k_new"], d_in["v_new"], d_in["k_cache"], d_in["v_cache"],
+                           d_in["slot_mapping"])
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        pkv.paged_attention_decode(out, d_in["q"], d_in["k_cache"], d_in["v_cache"],
+                                   d_in["block_tables"], d_in["seq_lens"], wl.max_seq_len,
+                                   wl.scale, workspace=ws)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    d_in = dict(dev)
+    d_in.update(meta)
+    step_bytes = (workloads.decode_algorithmic_bytes(wl) + workloads.write_bytes(wl) +
+                  workloads.copy_bytes(wl))
+    decode_bytes = workloads.decode_algorithmic_bytes(wl)
+    working_set = decode_bytes
+    flush = working_set < 8 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev_name) if flush else None
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step(d_in)
+    if flush:
+        scratch.fill_(1)
+    barrier()
+
+    def timed_region():
+        ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+        barrier()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank) as clocks:
+            torch.cuda.nvtx.range_push("timed_region")
+            t_start.record(stream)
+            for i in range(args.steps):
+                if flush:
+                    scratch.add_(1)  # evict the previous step's blocks from L2 (untimed below)
+                ev_step[i][0].record(stream)
+                step(d_in, ev_dec[i])
+                ev_step[i][1].record(stream)
+            t_end.record(stream)
+            torch.cuda.nvtx.range_pop()
+            barrier()
+        dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+        step_ms = [a.elapsed_time(b) for a, b in ev_step]
+        total_ms = sum(step_ms) if flush else t_start.elapsed_time(t_end)
+        return total_ms, dec_ms, clocks
+
+    total_ms, dec_ms, clocks = timed_region()
+    remeasured = False
+    if clocks.rejected():
+        total_ms, dec_ms, clocks = timed_region()
+        remeasured = True
+
+    # max over ranks (device-timed)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev_name)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms_max = float(t.item())
+    ms_per_step = total_ms_max / args.steps
+    value = world * step_bytes * args.steps / (total_ms_max * 1e-3) / 1e9
+    tokens_per_s = world * wl.B * args.steps / (total_ms_max * 1e-3)
+
+    # e2e through the public API: pinned host inputs -> device, step, output -> host.
+    host_in = {k: d_in[k].cpu().pin_memory() for k in
+               ("q", "k_new", "v_new", "block_tables", "seq_lens", "slot_mapping", "cow_pairs")}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for k, v in host_in.items()
+              if k != "cow_pairs" or has_cow)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, v in host_in.items():
+            if k != "cow_pairs" or has_cow:
+                d_in[k].copy_(v, non_blocking=True)
+        step(d_in)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 4)):
+        e2e_step()
+    if flush:
+        scratch.add_(1)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(10, args.steps // 4)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], dtype=torch.float64, device=dev_name)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_val = world * step_bytes / (float(e2e_ms.item()) * 1e-3) / 1e9
+
+    peak, peak_src = load_peaks()
+    dec_avg_ms = statistics.fmean(dec_ms)
+    achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
+    G = wl.G
+    kernel = ("paged_decode_kernel<MmaConsumer>" if wl.dtype == "bf16" and G >= 3
+              else "paged_decode_kernel<SimtConsumer>")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
+                "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
+                "decode_us": round(dec_avg_ms * 1e3, 2),
+                "algorithmic_bytes_per_launch": decode_bytes}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = host_pool_from(dev, wl)
+        n_seq = oracle_sample(wl, host, budget_rows=args.cpu_budget_rows)
+        dt, nbytes, tokens, cores = time_oracle(wl, host, n_seq)
+        cpu = {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+               "kind": "oracle",
+               "sample": f"decode of sequences 0..{n_seq - 1} of {wl.B} ({tokens} cached tokens, "
+                         f"{n_seq * wl.Hq} query rows), fp64, {dt:.2f} s",
+               "tokens_per_s": round(n_seq / dt, 3)}
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool, NaN in unused slots)",
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_of_8TBps_spec": round(100 * value / world / SPEC_HBM_GBS, 2),
+        "pct_of_measured_peak": round(100 * value / world / peak, 2),
+        "config": {"workload": args.config, "description": DESCR.get(args.config, args.config),
+                   "step": ("copy_blocks + " if has_cow else "") + "paged_kv_write + paged_attention_decode",
+                   "bytes_per_step": step_bytes,
+                   "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
+                          else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(float(e2e_ms.item()), 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if remeasured:
+        line["clocks"]["remeasured"] = True
+    return line
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle on this host's cores, each step a bounded sample
+    of the same workload."""
+    if rank != 0:
+        return None
+    wl = workloads.make(args.config)
+    host = workloads.host_tensors(wl) if wl.num_blocks * wl.block_bytes < (6 << 30) else None
+    if host is None:
+        raise SystemExit("workload too large for a host-side reference run")
+    n_seq = oracle_sample(wl, host, budget_rows=args.cpu_budget_rows // max(args.steps, 1))
+    for _ in range(args.warmup):
+        time_oracle(wl, host, max(1, n_seq // 8))
+    total_t, total_b, cores, tokens = 0.0, 0, 1, 0
+    for _ in range(args.steps):
+        dt, nb, tk, cores = time_oracle(wl, host, n_seq)
+        total_t += dt
+        total_b += nb
+        tokens += tk
+    val = total_b / total_t / 1e9
+    sample = f"decode of sequences 0..{n_seq - 1} of {wl.B} per step, fp64"
+    return {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.config, "description": DESCR.get(args.config, "")},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="mha", choices=sorted(DESCR))
+    ap.add_argument("--cpu-budget-rows", type=int, default=400_000_000,
+                    help="query-row x token budget of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local_rank}"))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

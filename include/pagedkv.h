@@ -1,0 +1,203 @@
+/*
+ * pagedkv.h: C ABI of libpagedkv.so, decode-step attention over a block-paged
+ * KV cache on NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages on paged attention; cited by title and section):
+ *   [Explained] "Paged Attention Explained: How LLMs Manage GPU Memory for
+ *               Faster AI Inference"
+ *   [Wiki]      "PagedAttention: paging the KV cache like an OS pages memory"
+ *   [Index]     "PagedAttention and KV Cache Compression: Optimizing LLM
+ *               Inference"
+ *
+ * Data layout (row-major, element type bf16 or fp32, identical for K and V):
+ *   k_cache, v_cache  [num_blocks][block_size][Hkv][D]   the block pool
+ *   block_tables      [B][max_blocks] int32               physical id of each
+ *                                                         logical block
+ *   seq_lens          [B] int32                           cached tokens per sequence
+ *   q, out            [B][Hq][D]                          one query per sequence
+ *   k, v (new tokens) [N][Hkv][D]
+ *   slot_mapping      [N] int64, slot = block * block_size + offset; < 0 skips
+ *   block_mapping     [P][2] int64, (src, dst) physical block ids
+ *
+ * Conventions shared by every call:
+ *   - Ownership: every pointer is caller-owned device memory (pointers that are
+ *     passed to a kernel must be device-accessible).  The library keeps no
+ *     pointer after the call returns.  Apart from the decode workspace, which
+ *     the caller provides, it allocates no device memory.
+ *   - Streams: every call enqueues its work on `stream` (NULL = the legacy
+ *     default stream) and returns without synchronising.
+ *   - Alignment: every data pointer must be 16-byte aligned.
+ *   - Errors: a call returns PKV_OK or a negative status.  It validates
+ *     arguments on the host before enqueueing anything, and on a validation
+ *     error nothing is enqueued.  Values that only the device sees (slots,
+ *     block ids, lengths) are range-checked in the kernels: an offending entry
+ *     is skipped or clamped, never dereferenced out of bounds, and its bit
+ *     is OR-ed into a device error word that pkv_device_errors() reads.
+ */
+#ifndef PAGEDKV_H_
+#define PAGEDKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *pkv_stream_t;
+
+/* Element type of q, k, v, out and both caches. */
+typedef enum { PKV_BF16 = 0, PKV_F32 = 1 } pkv_dtype;
+
+/* Status codes. */
+enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, bad dimension or dtype */
+    PKV_ERR_OUT_OF_RANGE = -2, /* a host-checkable size or bound is out of range */
+    PKV_ERR_WORKSPACE = -3,    /* decode workspace missing or too small */
+    PKV_ERR_CUDA = -4,         /* a CUDA call failed; see pkv_last_cuda_error() */
+    PKV_ERR_UNSUPPORTED = -5   /* valid but unsupported shape (head dim, block size, G) */
+};
+
+/* Device error bits (pkv_device_errors). */
+#define PKV_DEVERR_SLOT 0x1u     /* paged_kv_write skipped a slot >= num_blocks*block_size */
+#define PKV_DEVERR_SEQLEN 0x2u   /* a seq_len < 0, > max_blocks*block_size or > max_seq_len was clamped */
+#define PKV_DEVERR_BLOCK_ID 0x4u /* a block-table id outside [0, num_blocks) was read as zeros */
+#define PKV_DEVERR_COPY 0x8u     /* copy_blocks skipped a pair with an id outside [0, num_blocks) */
+#define PKV_DEVERR_TIMEOUT 0x10u /* a pipeline wait gave up after its time limit */
+
+/*
+ * paged_kv_write: the cache update.  [Explained] "Step 2: Allocate Blocks
+ * Dynamically" and the list of duties of a production implementation ("cache
+ * updates") in "Practical Example"; [Index] "5. Real-World Consequences" (a
+ * new token fills the current block; a new block only when it is full).
+ *
+ * For every n < N with s = slot_mapping[n] >= 0, row n of k and v
+ * (Hkv*D elements each) is copied bit for bit to k_cache and v_cache at
+ * block s / block_size, offset s % block_size.  Slots < 0 are skipped.
+ * Slots >= num_blocks*block_size are skipped and flag PKV_DEVERR_SLOT.
+ * Two tokens with the same slot race (one of them wins).
+ *   k, v            device [N][Hkv][D]
+ *   k_cache,v_cache device [num_blocks][block_size][Hkv][D], updated in place
+ *   slot_mapping    device [N] int64
+ * Requires Hkv*D*element size to be a multiple of 16 bytes.  N == 0 is a no-op.
+ */
+int paged_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
+                   const int64_t *slot_mapping, int64_t N, int Hkv, int D, int block_size,
+                   int64_t num_blocks, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * Partition length (tokens) that paged_attention_decode uses for these sizes:
+ * `partition_size` itself when it is > 0, otherwise the library's choice.
+ * The choice is a multiple of 16 and depends only on the arguments.
+ * Returns a negative status for invalid arguments.
+ */
+int paged_attention_decode_partition_size(int B, int Hkv, int max_seq_len, int block_size,
+                                          int partition_size);
+
+/*
+ * Workspace bytes paged_attention_decode needs for these sizes: 0 when every
+ * sequence fits in one partition.  It is a pure host function with no CUDA
+ * calls.  Returns 0 for invalid arguments (the call then reports the error).
+ */
+size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_seq_len,
+                                             int block_size, int partition_size);
+
+/*
+ * paged_attention_decode: single-query attention over the paged cache.
+ * The attention is ordinary softmax attention; only the storage layout
+ * differs ([Wiki] "How it works").  The kernel follows the block table to
+ * find each token's keys and values ([Explained] "Step 3: Maintain a Block
+ * Table", "Step 4: Retrieve Cached Data During Attention"; [Index] "4.
+ * Technical Depth").  Scores are accumulated with a running maximum and sum
+ * (online softmax, the tiling idea named in [Explained] "What Is the
+ * Difference Between PagedAttention and FlashAttention?").
+ *
+ * For b < B and h < Hq, with G = Hq / Hkv, kvh = h / G, L = seq_lens[b]:
+ *   K_t = k_cache[block_tables[b][t / block_size]][t % block_size][kvh]
+ *   V_t likewise, for t < L
+ *   out[b][h] = sum_t softmax_t(scale * q[b][h] . K_t) * V_t
+ * out[b][h] = 0 when L == 0.  Arithmetic is fp32; bf16 inputs are widened
+ * exactly and the result is rounded to nearest even.  Slots past L in the
+ * last block, and table entries past ceil(L / block_size), are never read.
+ *
+ * Long sequences are split into partitions of P tokens
+ * (paged_attention_decode_partition_size).  Each partition yields a partial
+ * (max, sum, weighted V), and the partials are merged with a log-sum-exp
+ * rescale in the same launch.
+ *
+ *   out             device [B][Hq][D], written
+ *   q               device [B][Hq][D]
+ *   k_cache,v_cache device [num_blocks][block_size][Hkv][D]
+ *   block_tables    device [B][max_blocks] int32
+ *   seq_lens        device [B] int32
+ *   max_seq_len     host upper bound of seq_lens (sets the partition grid
+ *                   without a device-to-host copy); a larger seq_len is
+ *                   clamped to it and flags PKV_DEVERR_SEQLEN
+ *   partition_size  0 = library choice, else a positive multiple of 16
+ *   workspace       device, >= paged_attention_decode_workspace_size(...)
+ *                   bytes, 256-byte aligned, ZERO-FILLED before its first
+ *                   use.  Each completed call leaves it ready for the next
+ *                   one (its counters are back at zero).  Two calls that
+ *                   share a workspace must not overlap on the GPU.  It may be
+ *                   NULL when the size is 0.
+ * Supported: bf16 with D in {64, 128, 256}; fp32 with D in {64, 128};
+ * block_size a multiple of 16 up to 256; G = Hq / Hkv <= 16 (bf16) or <= 8
+ * (fp32); num_blocks * block_size < 2^31.
+ */
+int paged_attention_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_tables, int max_blocks, const int32_t *seq_lens,
+                           int max_seq_len, int B, int Hq, int Hkv, int D, int block_size,
+                           int64_t num_blocks, float scale, pkv_dtype dtype,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           pkv_stream_t stream);
+
+/*
+ * copy_blocks: block-granularity copy-on-write copies.  Physical blocks are
+ * reference-counted and shared between requests or decode branches, and a
+ * shared block that must be modified is first copied ([Wiki] "How it works";
+ * [Index] "Complex Decoding (Beam Search & Parallel Sampling)", glossary
+ * "Copy-on-Write").  Deciding which blocks to copy is the caller's job.
+ *
+ * For each pair i < P: k_cache[dst] = k_cache[src] and v_cache[dst] =
+ * v_cache[src], whole blocks of block_bytes bytes, bit for bit.  The dst ids
+ * must be distinct and no dst may also be a src (otherwise the result
+ * depends on order).  Pairs with an id outside [0, num_blocks) are skipped
+ * and flag PKV_DEVERR_COPY.
+ *   k_cache,v_cache device pools of num_blocks blocks of block_bytes each
+ *   block_mapping   device [P][2] int64 (src, dst)
+ *   block_bytes     block_size*Hkv*D*element size, a multiple of 16
+ */
+int copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int64_t P,
+                int64_t block_bytes, int64_t num_blocks, pkv_stream_t stream);
+
+/* Short English text for a status code (static storage). */
+const char *pkv_status_string(int status);
+
+/* The cudaError_t of the last PKV_ERR_CUDA returned on this host thread. */
+int pkv_last_cuda_error(void);
+
+/*
+ * Reads the device error word of the current device into *bits, and clears it
+ * when `clear` is non-zero.  This synchronises with the device.
+ */
+int pkv_device_errors(uint32_t *bits, int clear);
+
+/*
+ * Arithmetic units used by paged_attention_decode, set for the whole process
+ * (for testing and measuring both kernels):
+ *   PKV_PATH_AUTO          bf16 with G >= 3 on tensor cores, all else on CUDA cores;
+ *   PKV_PATH_CUDA_CORES    fp32 FMAs whenever G <= 8;
+ *   PKV_PATH_TENSOR_CORES  warp-level bf16 MMA for every bf16 call.
+ * fp32 always runs on CUDA cores.  Returns the previous mode, or
+ * PKV_ERR_INVALID_ARG.  The results of both kernels satisfy the same bounds.
+ */
+enum { PKV_PATH_AUTO = 0, PKV_PATH_CUDA_CORES = 1, PKV_PATH_TENSOR_CORES = 2 };
+int pkv_set_decode_path(int mode);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H_ */

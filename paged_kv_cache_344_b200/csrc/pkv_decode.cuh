@@ -1,0 +1,614 @@
+// Decode-step attention over a block-paged KV cache (sm_100a).
+//
+// What is computed: for sequence b and query head h (KV head kvh = h / G),
+//   out[b][h] = sum_t softmax_t(scale * q[b][h] . K_t) V_t,  t < seq_lens[b],
+// with K_t, V_t found through the block table: logical block t / block_size,
+// offset t % block_size ("Paged Attention Explained", Step 3 and Step 4;
+// "PagedAttention: paging the KV cache like an OS pages memory", How it works:
+// the attention is ordinary softmax attention, only the layout changes).
+//
+// How (B200 design):
+//  * one CTA per (kvh, partition, b); the G query heads of a KV head share
+//    every K/V byte read, so the cache is read once per (b, kvh);
+//  * K/V arrive by TMA: a 3-D tensor map over [num_blocks*bs][Hkv][D] fetches
+//    one 16-token slab of one KV head per box; each consumer warp owns a ring
+//    of stages and refills it itself, so no CTA-wide barrier sits in the loop;
+//  * the block-table walk (the "pointer chase") is taken off the critical path:
+//    each warp keeps the physical ids of its next 32..64 stages in registers;
+//  * online softmax in fp32 (running max and sum, exp2 with the scale folded
+//    into log2 units), per warp; warps and then partitions are merged with a
+//    log-sum-exp rescale;
+//  * grouped heads (G > 2, bf16) run the score and PV products on the tensor
+//    cores with a warp-level m16n8k16 MMA: tokens are M, the G heads are N
+//    (padded to 8), D is K; PV computes O^T = V^T P^T with P transposed in
+//    registers by movmatrix.  Smaller G and fp32 use CUDA-core FMAs;
+//  * a sequence split into several partitions writes partial (max, sum,
+//    weighted V) to the workspace; the CTA that finishes last for a
+//    (b, kvh) -- found with an atomic ticket, no spinning -- merges them.
+#pragma once
+
+#include "pkv_ptx.cuh"
+
+namespace pkv {
+
+constexpr int kStageTokens = 16;  // tokens per TMA box / pipeline stage
+constexpr int kWarps = 4;         // consumer warps per CTA
+constexpr uint32_t kFull = 0xffffffffu;
+
+__device__ uint32_t g_device_errors;  // OR of PKV_DEVERR_* bits
+
+__device__ __forceinline__ void flag_error(uint32_t bits) { atomicOr(&g_device_errors, bits); }
+
+struct DecodeParams {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  float* ws_acc;       // [B*Hkv*max_parts*G][D]
+  float2* ws_ml;       // [B*Hkv*max_parts*G] (max in log2 units, sum)
+  uint32_t* ws_count;  // [B*Hkv] finished-partition tickets
+  int max_blocks;
+  int max_seq_len;
+  int Hq;
+  int Hkv;
+  int G;
+  int bs;
+  int part_tokens;
+  int max_parts;
+  int num_blocks;
+  float scale_log2;  // scale * log2(e)
+};
+
+template <typename T>
+__device__ __forceinline__ T to_out(float x);
+template <>
+__device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ float to_out<float>(float x) {
+  return x;
+}
+
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4& w, float* f);
+template <>
+__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4& w, float* f) {
+  f[0] = bf16_lo(w.x); f[1] = bf16_hi(w.x); f[2] = bf16_lo(w.y); f[3] = bf16_hi(w.y);
+  f[4] = bf16_lo(w.z); f[5] = bf16_hi(w.z); f[6] = bf16_lo(w.w); f[7] = bf16_hi(w.w);
+}
+template <>
+__device__ __forceinline__ void unpack16<float>(const uint4& w, float* f) {
+  f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+  f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+}
+
+// Loads N consecutive elements of type T from shared memory as floats.
+template <typename T, int N>
+__device__ __forceinline__ void load_row_slice(const uint8_t* src, float* f) {
+  constexpr int BYTES = N * (int)sizeof(T);
+  if constexpr (BYTES == 16) {
+    unpack16<T>(*reinterpret_cast<const uint4*>(src), f);
+  } else if constexpr (BYTES == 8) {
+    const uint2 w = *reinterpret_cast<const uint2*>(src);
+    if constexpr (sizeof(T) == 2) {
+      f[0] = bf16_lo(w.x); f[1] = bf16_hi(w.x); f[2] = bf16_lo(w.y); f[3] = bf16_hi(w.y);
+    } else {
+      f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+    }
+  } else if constexpr (BYTES == 4) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+    if constexpr (sizeof(T) == 2) {
+      f[0] = bf16_lo(w); f[1] = bf16_hi(w);
+    } else {
+      f[0] = __uint_as_float(w);
+    }
+  } else {
+    static_assert(BYTES == 32, "unsupported slice");
+    unpack16<T>(*reinterpret_cast<const uint4*>(src), f);
+    unpack16<T>(*reinterpret_cast<const uint4*>(src + 16), f + 16 / sizeof(T));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core consumer: one warp processes a 16-token stage.  QK: LPT lanes per
+// token, each lane two 16-byte chunks of the K row; PV: each lane D/32
+// consecutive dims of every V row.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int GMAX>
+struct SimtConsumer {
+  static constexpr int ES = sizeof(T);
+  static constexpr int ROWB = D * ES;
+  static constexpr int CH = ROWB / 16;
+  static constexpr int LPT = CH / 2;
+  static constexpr int TPI = 32 / LPT;
+  static constexpr int ITERS = kStageTokens / TPI;
+  static constexpr int EPC = 16 / ES;
+  static constexpr int DPL = D / 32;
+  static constexpr int kTileBytes = kStageTokens * ROWB;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = ROWB <= 128 ? 6 : (ROWB <= 256 ? 3 : 2);
+  static constexpr int GP = GMAX;
+  static constexpr bool kSwizzle = false;
+  static_assert(LPT >= 1 && LPT <= 32 && TPI * LPT == 32, "bad lane split");
+
+  float qv[GMAX][2][EPC];
+  float m[GMAX], l[GMAX], acc[GMAX][DPL];
+
+  __device__ __forceinline__ void init(const DecodeParams& p, int b, int kvh, int lane) {
+    const int sub = lane % LPT;
+    const T* q = reinterpret_cast<const T*>(p.q);
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      if (g < p.G) {
+        const T* row = q + ((size_t)b * p.Hq + (size_t)kvh * p.G + g) * D;
+        unpack16<T>(*reinterpret_cast<const uint4*>(row + sub * EPC), qv[g][0]);
+        unpack16<T>(*reinterpret_cast<const uint4*>(row + (sub + LPT) * EPC), qv[g][1]);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) {
+          qv[g][0][e] *= p.scale_log2;
+          qv[g][1][e] *= p.scale_log2;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) qv[g][0][e] = qv[g][1][e] = 0.f;
+      }
+      m[g] = -INFINITY;
+      l[g] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[g][e] = 0.f;
+    }
+  }
+
+  static __device__ __forceinline__ void load_stage(uint8_t* st, const CUtensorMap* tk,
+                                                    const CUtensorMap* tv, uint64_t* bar,
+                                                    int kvh, int row, uint64_t pol) {
+    tma_load_3d(st, tk, bar, 0, kvh, row, pol);
+    tma_load_3d(st + kTileBytes, tv, bar, 0, kvh, row, pol);
+  }
+
+  __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane) {
+    const uint8_t* sk = st;
+    const uint8_t* sv = st + kTileBytes;
+    const int sub = lane % LPT;
+    const int tg = lane / LPT;
+    float s[ITERS][GMAX];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+      const int tok = it * TPI + tg;
+      float k0[EPC], k1[EPC];
+      unpack16<T>(*reinterpret_cast<const uint4*>(sk + tok * ROWB + sub * 16), k0);
+      unpack16<T>(*reinterpret_cast<const uint4*>(sk + tok * ROWB + (sub + LPT) * 16), k1);
+#pragma unroll
+      for (int g = 0; g < GMAX; ++g) {
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) part = fmaf(qv[g][0][e], k0[e], part);
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) part = fmaf(qv[g][1][e], k1[e], part);
+#pragma unroll
+        for (int off = LPT / 2; off >= 1; off /= 2) part += __shfl_xor_sync(kFull, part, off);
+        s[it][g] = (tok < n_valid) ? part : -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      float mx = s[0][g];
+#pragma unroll
+      for (int it = 1; it < ITERS; ++it) mx = fmaxf(mx, s[it][g]);
+#pragma unroll
+      for (int off = LPT; off < 32; off *= 2) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, off));
+      const float m_new = fmaxf(m[g], mx);
+      const float alpha = exp2f(m[g] - m_new);
+      m[g] = m_new;
+      float sum = 0.f;
+#pragma unroll
+      for (int it = 0; it < ITERS; ++it) {
+        s[it][g] = exp2f(s[it][g] - m_new);
+        sum += s[it][g];
+      }
+#pragma unroll
+      for (int off = LPT; off < 32; off *= 2) sum += __shfl_xor_sync(kFull, sum, off);
+      l[g] = l[g] * alpha + sum;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[g][e] *= alpha;
+    }
+#pragma unroll
+    for (int t = 0; t < kStageTokens; ++t) {
+      if (t < n_valid) {
+        float v[DPL];
+        load_row_slice<T, DPL>(sv + t * ROWB + lane * DPL * ES, v);
+#pragma unroll
+        for (int g = 0; g < GMAX; ++g) {
+          const float pt = __shfl_sync(kFull, s[t / TPI][g], (t % TPI) * LPT);
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc[g][e] = fmaf(pt, v[e], acc[g][e]);
+        }
+      }
+    }
+  }
+
+  // Per-warp state -> shared memory: m[GP], l[GP], acc[GP][D].
+  __device__ __forceinline__ void store_state(float* dst, int lane) const {
+#pragma unroll
+    for (int g = 0; g < GMAX; ++g) {
+      if (lane == 0) {
+        dst[g] = m[g];
+        dst[GP + g] = l[g];
+      }
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) dst[2 * GP + g * D + lane * DPL + e] = acc[g][e];
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Tensor-core consumer (bf16): S[t][g] = K[t][:] . Q[g][:] with tokens as M,
+// heads as N; O^T[d][g] += V^T[d][t] P[t][g].  K/V tiles arrive with the TMA
+// 128-byte swizzle (D/64 sub-tiles of 16 rows x 128 B), which keeps the
+// ldmatrix row reads free of bank conflicts.
+// ---------------------------------------------------------------------------
+template <int D, int NT>
+struct MmaConsumer {
+  static constexpr int SUB = D / 64;
+  static constexpr int kSubBytes = kStageTokens * 128;
+  static constexpr int kTileBytes = SUB * kSubBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = D <= 64 ? 6 : (D <= 128 ? 3 : 2);
+  static constexpr int KS = D / 16;
+  static constexpr int MT = D / 16;
+  static constexpr int GP = 8 * NT;
+  static constexpr bool kSwizzle = true;
+
+  uint32_t qf[NT][KS][2];
+  float m[NT][2], l[NT][2];
+  float o[NT][MT][4];
+  float scale_log2;
+
+  __device__ __forceinline__ void init(const DecodeParams& p, int b, int kvh, int lane) {
+    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+    scale_log2 = p.scale_log2;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 8 + lane / 4;
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(
+          q + ((size_t)b * p.Hq + (size_t)kvh * p.G + (g < p.G ? g : 0)) * D);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int d0 = ks * 16 + 2 * (lane % 4);
+        qf[nt][ks][0] = g < p.G ? row[d0 / 2] : 0u;
+        qf[nt][ks][1] = g < p.G ? row[(d0 + 8) / 2] : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m[nt][j] = -INFINITY;
+        l[nt][j] = 0.f;
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[nt][mt][j] = 0.f;
+    }
+  }
+
+  static __device__ __forceinline__ void load_stage(uint8_t* st, const CUtensorMap* tk,
+                                                    const CUtensorMap* tv, uint64_t* bar,
+                                                    int kvh, int row, uint64_t pol) {
+#pragma unroll
+    for (int sb = 0; sb < SUB; ++sb) {
+      tma_load_3d(st + sb * kSubBytes, tk, bar, sb * 64, kvh, row, pol);
+      tma_load_3d(st + kTileBytes + sb * kSubBytes, tv, bar, sb * 64, kvh, row, pol);
+    }
+  }
+
+  // Byte offset of (row, 16-byte chunk) inside a swizzled 16x128 B sub-tile.
+  static __device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+  }
+
+  __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane) {
+    const uint32_t sk = smem_u32(st);
+    const uint32_t sv = sk + kTileBytes;
+    const int mi = lane / 8, rr = lane % 8;
+
+    // Scores: S = K Q^T, one m16n8k16 per (k-step, head tile).
+    float s[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[nt][j] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int row = rr + (mi & 1) * 8;
+      const int chunk = (ks % 4) * 2 + (mi >> 1);
+      uint32_t a[4];
+      ldmatrix_x4(sk + (ks / 4) * kSubBytes + swz(row, chunk), a[0], a[1], a[2], a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+    }
+
+    // Invalid tail slots of the last stage hold anything (even NaN): their
+    // scores are replaced by -inf, and their V rows are zeroed before the PV
+    // product so that 0 * NaN cannot reach the accumulator.
+    if (n_valid < kStageTokens) {
+      uint4* vz = reinterpret_cast<uint4*>(st + kTileBytes);
+      const int nvec = (kStageTokens - n_valid) * 8;  // 128-byte rows, per sub-tile
+#pragma unroll
+      for (int sb = 0; sb < SUB; ++sb)
+        for (int i = lane; i < nvec; i += 32)
+          vz[sb * (kSubBytes / 16) + n_valid * 8 + i] = make_uint4(0u, 0u, 0u, 0u);
+      fence_proxy_async_smem();
+      __syncwarp();
+    }
+
+    const int t0 = lane / 4;
+    uint32_t pb[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float x[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = t0 + (j >> 1) * 8;
+        x[j] = (t < n_valid) ? s[nt][j] * scale_log2 : -INFINITY;
+      }
+      float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off *= 2) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+      }
+      const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+      const float al0 = exp2f(m[nt][0] - mn0), al1 = exp2f(m[nt][1] - mn1);
+      m[nt][0] = mn0;
+      m[nt][1] = mn1;
+      x[0] = exp2f(x[0] - mn0);
+      x[1] = exp2f(x[1] - mn1);
+      x[2] = exp2f(x[2] - mn0);
+      x[3] = exp2f(x[3] - mn1);
+      float sum0 = x[0] + x[2], sum1 = x[1] + x[3];
+#pragma unroll
+      for (int off = 4; off < 32; off *= 2) {
+        sum0 += __shfl_xor_sync(kFull, sum0, off);
+        sum1 += __shfl_xor_sync(kFull, sum1, off);
+      }
+      l[nt][0] = l[nt][0] * al0 + sum0;
+      l[nt][1] = l[nt][1] * al1 + sum1;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        o[nt][mt][0] *= al0;
+        o[nt][mt][1] *= al1;
+        o[nt][mt][2] *= al0;
+        o[nt][mt][3] *= al1;
+      }
+      // P (rows t, cols g) -> B fragment of P with k = t, n = g.
+      pb[nt][0] = movmatrix_trans(pack_bf16x2(x[0], x[1]));
+      pb[nt][1] = movmatrix_trans(pack_bf16x2(x[2], x[3]));
+    }
+
+    // O^T += V^T P: one m16n8k16 per (16-dim tile, head tile).
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int t = (mi >> 1) * 8 + rr;
+      const int d0 = mt * 16 + (mi & 1) * 8;
+      uint32_t a[4];
+      ldmatrix_x4_trans(sv + (d0 / 64) * kSubBytes + swz(t, (d0 % 64) / 8), a[0], a[1], a[2],
+                        a[3]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
+    }
+  }
+
+  __device__ __forceinline__ void store_state(float* dst, int lane) const {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int g = nt * 8 + 2 * (lane % 4);
+      if (lane < 4) {
+        dst[g] = m[nt][0];
+        dst[g + 1] = m[nt][1];
+        dst[GP + g] = l[nt][0];
+        dst[GP + g + 1] = l[nt][1];
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int d = mt * 16 + lane / 4;
+        dst[2 * GP + g * D + d] = o[nt][mt][0];
+        dst[2 * GP + (g + 1) * D + d] = o[nt][mt][1];
+        dst[2 * GP + g * D + d + 8] = o[nt][mt][2];
+        dst[2 * GP + (g + 1) * D + d + 8] = o[nt][mt][3];
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// The kernel skeleton shared by both consumers.
+// ---------------------------------------------------------------------------
+template <class C>
+struct DecodeSmem {
+  static constexpr int kRingBytes = C::kStages * C::kStageBytes;
+  static constexpr size_t kBytes =
+      1024 /*alignment slack*/ + (size_t)kWarps * kRingBytes + kWarps * C::kStages * 8;
+};
+
+template <class C, typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int kRing = DecodeSmem<C>::kRingBytes;
+  static_assert(kRing >= (2 * C::GP + C::GP * D) * 4, "state does not fit in the ring");
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kRing);
+  __shared__ float s_M[16], s_den[16];
+  __shared__ int s_last;
+
+  const int kvh = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = p.G;
+  const int P = p.part_tokens;
+
+  // After a pipeline timeout anywhere, later CTAs stop at once instead of waiting too.
+  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  int L = p.seq_lens[b];
+  const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
+  if (L < 0 || L > Lcap) {
+    if (threadIdx.x == 0 && part == 0 && kvh == 0) flag_error(PKV_DEVERR_SEQLEN);
+    L = L < 0 ? 0 : Lcap;
+  }
+  const int nparts = (L + P - 1) / P;
+  T* out = reinterpret_cast<T*>(p.out) + ((size_t)b * p.Hq + (size_t)kvh * G) * D;
+  if (L == 0) {
+    if (part == 0)
+      for (int i = threadIdx.x; i < G * D; i += blockDim.x) out[i] = to_out<T>(0.f);
+    return;
+  }
+  if (part >= nparts) return;
+
+  const int t_begin = part * P;
+  const int t_end = min(L, t_begin + P);
+  const int n_st = (t_end - t_begin + kStageTokens - 1) / kStageTokens;
+  const int n_w = n_st > warp ? (n_st - warp + kWarps - 1) / kWarps : 0;
+
+  uint8_t* ring = smem + warp * kRing;
+  uint64_t* wbar = bars + warp * C::kStages;
+  if (lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+#pragma unroll
+    for (int s = 0; s < C::kStages; ++s) mbar_init(&wbar[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  const uint64_t pol = l2_policy_evict_first();
+  const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks;
+  auto stage_id = [&](int k) -> int {
+    const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
+    return bt_row[t0 / p.bs];
+  };
+  // Physical ids of this warp's stages win_base .. win_base+63 (one per lane, two windows).
+  int win_base = 0;
+  int win0 = lane < n_w ? stage_id(lane) : -1;
+  int win1 = 32 + lane < n_w ? stage_id(32 + lane) : -1;
+
+  auto issue = [&](int k) {
+    if (k - win_base >= 32) {
+      win0 = win1;
+      win_base += 32;
+      win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane) : -1;
+    }
+    const int rel = k - win_base;
+    const int id = __shfl_sync(kFull, rel < 32 ? win0 : win1, rel & 31);
+    if (lane == 0) {
+      const int s = k % C::kStages;
+      const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
+      int row;
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PKV_DEVERR_BLOCK_ID);
+        row = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
+      } else {
+        row = id * p.bs + t0 % p.bs;
+      }
+      mbar_arrive_expect_tx(&wbar[s], C::kStageBytes);
+      C::load_stage(ring + s * C::kStageBytes, &tmK, &tmV, &wbar[s], kvh, row, pol);
+    }
+  };
+
+  const int n_pro = n_w < C::kStages ? n_w : C::kStages;
+  for (int k = 0; k < n_pro; ++k) issue(k);
+
+  C c;
+  c.init(p, b, kvh, lane);
+
+  for (int k = 0; k < n_w; ++k) {
+    const int s = k % C::kStages;
+    const uint32_t parity = (uint32_t)((k / C::kStages) & 1);
+    const bool ok = mbar_wait_bounded(&wbar[s], parity);
+    if (__any_sync(kFull, !ok)) {
+      // Give up: flag it, wait (bounded) for the other loads in flight, stop.
+      if (lane == 0) flag_error(PKV_DEVERR_TIMEOUT);
+      for (int j = k; j < n_w && j < k + C::kStages; ++j)
+        mbar_wait_bounded(&wbar[j % C::kStages], (uint32_t)((j / C::kStages) & 1));
+      break;
+    }
+    const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
+    const int n_valid = min(kStageTokens, t_end - t0);
+    c.consume(ring + s * C::kStageBytes, n_valid, lane);
+    __syncwarp();
+    if (k + C::kStages < n_w) issue(k + C::kStages);
+  }
+
+  // Merge the warps' states (each in its own, now idle, ring).
+  c.store_state(reinterpret_cast<float*>(ring), lane);
+  __syncthreads();
+  constexpr int GP = C::GP;
+  const bool split = nparts > 1;
+  const size_t unit = (size_t)b * p.Hkv + kvh;
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w)
+      M = fmaxf(M, reinterpret_cast<const float*>(smem + w * kRing)[g]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float* st = reinterpret_cast<const float*>(smem + w * kRing);
+      const float f = exp2f(st[g] - M);
+      num = fmaf(f, st[2 * GP + g * D + d], num);
+      den = fmaf(f, st[GP + g], den);
+    }
+    if (!split) {
+      out[idx] = to_out<T>(num / den);
+    } else {
+      const size_t u = (unit * p.max_parts + part) * G + g;
+      p.ws_acc[u * D + d] = num;
+      if (d == 0) p.ws_ml[u] = make_float2(M, den);
+    }
+  }
+  if (!split) return;
+
+  // Partition merge: the last CTA of this (b, kvh) to finish does it.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atomicAdd(&p.ws_count[unit], 1u);
+    s_last = (prev == (uint32_t)(nparts - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const size_t base = unit * p.max_parts * G;
+  for (int g = warp; g < G; g += kWarps) {
+    float M = -INFINITY;
+    for (int q = lane; q < nparts; q += 32) M = fmaxf(M, __ldcg(&p.ws_ml[base + (size_t)q * G + g]).x);
+#pragma unroll
+    for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+    float den = 0.f;
+    for (int q = lane; q < nparts; q += 32) {
+      const float2 ml = __ldcg(&p.ws_ml[base + (size_t)q * G + g]);
+      den += exp2f(ml.x - M) * ml.y;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
+    if (lane == 0) {
+      s_M[g] = M;
+      s_den[g] = den;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int g = idx / D, d = idx % D;
+    const float M = s_M[g];
+    float num = 0.f;
+    for (int q = 0; q < nparts; ++q) {
+      const size_t u = base + (size_t)q * G + g;
+      num = fmaf(exp2f(__ldcg(&p.ws_ml[u]).x - M), __ldcg(&p.ws_acc[u * D + d]), num);
+    }
+    out[idx] = to_out<T>(num / s_den[g]);
+  }
+  if (threadIdx.x == 0) p.ws_count[unit] = 0u;
+}
+
+}  // namespace pkv

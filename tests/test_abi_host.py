@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI: the library loads, exports every function its header
+declares, and rejects bad arguments on the host before enqueueing anything.  No kernel
+runs here.  The invalid calls use fake device addresses, so these tests are skipped when
+a GPU is visible: if a check ever let one of them through, it must not reach a kernel."""
+import ctypes
+
+import pytest
+
+import paged_kv_cache_344_b200 as pkv
+from paged_kv_cache_344_b200 import build
+
+ERR_ARG, ERR_RANGE, ERR_WS, ERR_CUDA, ERR_UNSUP = -1, -2, -3, -4, -5
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return pkv.lib()
+
+
+def _no_gpu():
+    import torch
+    return not torch.cuda.is_available()
+
+
+host_only = pytest.mark.skipif(not _no_gpu(), reason="fake-pointer calls run only without a GPU")
+
+
+def test_exports_every_declared_symbol(lib):
+    names = pkv.declared_functions()
+    assert {"paged_kv_write", "paged_attention_decode", "copy_blocks",
+            "paged_attention_decode_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/pagedkv.h but not exported"
+
+
+def test_status_strings(lib):
+    for code in (0, ERR_ARG, ERR_RANGE, ERR_WS, ERR_CUDA, ERR_UNSUP, 99):
+        assert lib.pkv_status_string(code)
+
+
+def test_partition_and_workspace_sizes(lib):
+    # requested partition sizes are honoured; the automatic one is a multiple of 16
+    assert pkv.paged_attention_decode_partition_size(8, 8, 131073, 16, 512) == 512
+    for B, Hkv, L in [(64, 40, 2049), (256, 8, 4097), (8, 8, 131073), (128, 8, 1281), (4, 4, 34)]:
+        P = pkv.paged_attention_decode_partition_size(B, Hkv, L, 16, 0)
+        assert P > 0 and P % 16 == 0
+    with pytest.raises(pkv.PagedKVError):
+        pkv.paged_attention_decode_partition_size(8, 8, 100, 16, 24)  # not a multiple of 16
+    # a single partition needs no workspace
+    assert pkv.paged_attention_decode_workspace_size(4, 4, 4, 64, 34, 16, 0) == 0
+    assert pkv.paged_attention_decode_workspace_size(8, 64, 8, 128, 1000, 16, 1024) == 0
+    # split partitions: counters + (max, sum) + D floats per (b, kvh, part, head)
+    ws = pkv.paged_attention_decode_workspace_size(8, 64, 8, 128, 131073, 16, 2048)
+    parts = -(-131073 // 2048)
+    assert ws >= 8 * 8 * parts * 8 * (128 + 2) * 4
+    assert ws <= 8 * 8 * parts * 8 * (128 + 2) * 4 + 4096
+    assert pkv.paged_attention_decode_workspace_size(8, 63, 8, 128, 1000, 16, 0) == 0  # invalid
+
+
+def _decode(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, mb=8, sl=FAKE, msl=100, B=2, Hq=8, Hkv=2,
+             D=128, bs=16, nb=64, scale=0.1, dt=0, part=0, ws=None, wsb=0)
+    a.update(kw)
+    return lib.paged_attention_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["mb"], a["sl"],
+                                      a["msl"], a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"],
+                                      a["nb"], a["scale"], a["dt"], a["part"], a["ws"], a["wsb"],
+                                      None)
+
+
+@host_only
+def test_decode_rejects_bad_arguments(lib):
+    assert _decode(lib, out=None) == ERR_ARG
+    assert _decode(lib, q=FAKE + 8) == ERR_ARG  # misaligned
+    assert _decode(lib, Hq=7) == ERR_ARG  # Hq % Hkv != 0
+    assert _decode(lib, Hkv=0) == ERR_ARG
+    assert _decode(lib, dt=7) == ERR_ARG
+    assert _decode(lib, scale=float("nan")) == ERR_ARG
+    assert _decode(lib, part=24) == ERR_ARG
+    assert _decode(lib, D=96) == ERR_UNSUP
+    assert _decode(lib, D=256, dt=1) == ERR_UNSUP
+    assert _decode(lib, bs=8) == ERR_UNSUP
+    assert _decode(lib, Hq=64, Hkv=2) == ERR_UNSUP  # G = 32
+    assert _decode(lib, msl=8 * 16 + 1) == ERR_RANGE
+    assert _decode(lib, nb=(1 << 31) // 16) == ERR_RANGE
+    # needs a workspace (split into partitions)
+    assert _decode(lib, msl=128, part=16) == ERR_WS
+    assert _decode(lib, msl=128, part=16, ws=FAKE, wsb=16) == ERR_WS
+    assert _decode(lib, msl=128, part=16, ws=FAKE + 16, wsb=1 << 20) == ERR_WS  # misaligned
+    # an empty batch is a no-op that succeeds without touching the device
+    assert _decode(lib, B=0) == 0
+
+
+@host_only
+def test_write_and_copy_reject_bad_arguments(lib):
+    w = lambda **kw: lib.paged_kv_write(kw.get("k", FAKE), FAKE, FAKE, FAKE, kw.get("slots", FAKE),
+                                        kw.get("N", 4), kw.get("Hkv", 8), kw.get("D", 128), 16,
+                                        kw.get("nb", 64), kw.get("dt", 0), None)
+    assert w(k=None) == ERR_ARG
+    assert w(k=FAKE + 4) == ERR_ARG
+    assert w(slots=FAKE + 4) == ERR_ARG
+    assert w(N=-1) == ERR_ARG
+    assert w(dt=3) == ERR_ARG
+    assert w(Hkv=1, D=3) == ERR_UNSUP  # row of 6 bytes
+    assert w(N=0) == 0
+    c = lambda **kw: lib.copy_blocks(kw.get("k", FAKE), FAKE, kw.get("m", FAKE), kw.get("P", 3),
+                                     kw.get("bb", 32768), kw.get("nb", 64), None)
+    assert c(k=None) == ERR_ARG
+    assert c(m=FAKE + 4) == ERR_ARG
+    assert c(bb=24) == ERR_UNSUP
+    assert c(P=-1) == ERR_ARG
+    assert c(nb=0) == ERR_ARG
+    assert c(P=0) == 0
+
+
+def test_decode_path_selector(lib):
+    old = pkv.set_decode_path(pkv.PKV_PATH_TENSOR_CORES)
+    assert pkv.set_decode_path(pkv.PKV_PATH_CUDA_CORES) == pkv.PKV_PATH_TENSOR_CORES
+    assert pkv.set_decode_path(old) == pkv.PKV_PATH_CUDA_CORES
+    with pytest.raises(pkv.PagedKVError):
+        pkv.set_decode_path(9)
