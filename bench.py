@@ -209,6 +209,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev_name = f"cuda:{local_rank}"
+    pkv.set_decode_path({"auto": pkv.PKV_PATH_AUTO, "cuda_cores": pkv.PKV_PATH_CUDA_CORES,
+                         "tensor_cores": pkv.PKV_PATH_TENSOR_CORES}[args.path])
     wl = workloads.make(args.config)
     dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
     meta = {
@@ -218,7 +220,9 @@ def run_ours(args, rank, world, local_rank):
         "cow_pairs": torch.from_numpy(wl.cow_pairs).to(dev_name),
     }
     ws_bytes = pkv.paged_attention_decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D,
-                                                         wl.max_seq_len, wl.bs, 0)
+                                                         wl.max_seq_len, wl.bs, args.partition)
+    part = pkv.paged_attention_decode_partition_size(wl.B, wl.Hkv, wl.max_seq_len, wl.bs,
+                                                     args.partition)
     ws = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev_name)
     out = torch.empty_like(dev["q"])
     has_cow = len(wl.cow_pairs) > 0
@@ -236,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
             ev_pair[0].record(stream)
         pkv.paged_attention_decode(out, d_in["q"], d_in["k_cache"], d_in["v_cache"],
                                    d_in["block_tables"], d_in["seq_lens"], wl.max_seq_len,
-                                   wl.scale, workspace=ws)
+                                   wl.scale, workspace=ws, partition_size=args.partition)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
@@ -336,8 +340,8 @@ def run_ours(args, rank, world, local_rank):
     dec_avg_ms = statistics.fmean(dec_ms)
     achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
     G = wl.G
-    kernel = ("paged_decode_kernel<MmaConsumer>" if wl.dtype == "bf16" and G >= 3
-              else "paged_decode_kernel<SimtConsumer>")
+    tc = wl.dtype == "bf16" and (args.path == "tensor_cores" or (args.path == "auto" and G >= 3))
+    kernel = "paged_decode_kernel<MmaConsumer>" if tc else "paged_decode_kernel<SimtConsumer>"
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
                 "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
@@ -369,7 +373,8 @@ def run_ours(args, rank, world, local_rank):
                    "bytes_per_step": step_bytes,
                    "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
                           else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "decode_path": args.path, "partition_tokens": part},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -424,6 +429,10 @@ def main():
     ap.add_argument("--cpu-budget-rows", type=int, default=400_000_000,
                     help="query-row x token budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["auto", "cuda_cores", "tensor_cores"], default="auto",
+                    help="decode kernel family (library default: auto)")
+    ap.add_argument("--partition", type=int, default=0,
+                    help="decode partition length in tokens (0 = library choice)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -175,7 +175,8 @@ int copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int6
 /* Short English text for a status code (static storage). */
 const char *pkv_status_string(int status);
 
-/* The cudaError_t of the last PKV_ERR_CUDA returned on this host thread. */
+/* The cudaError_t of the last PKV_ERR_CUDA returned on this host thread
+ * (100000 + CUresult when encoding a TMA tensor map failed). */
 int pkv_last_cuda_error(void);
 
 /*

@@ -63,14 +63,17 @@ int make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t r
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  if (r != CUDA_SUCCESS) {  // reported as 100000 + the driver's CUresult
+    g_last_cuda_error = 100000 + static_cast<int>(r);
+    return PKV_ERR_CUDA;
+  }
   return PKV_OK;
 }
 
-// Raises the dynamic shared-memory limit of a kernel once per device.
+// Raises the dynamic shared-memory limit of a kernel once per device.  `done`
+// must be distinct for every kernel (all decode kernels share one C++ type).
 template <typename Kernel>
-int ensure_smem(Kernel kernel, size_t bytes) {
-  static std::atomic<uint64_t> done{0};
+int ensure_smem(Kernel kernel, size_t bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -128,7 +131,8 @@ int launch_decode(const pkv::DecodeParams& p, int B, const CUtensorMap& mk, cons
                   cudaStream_t stream) {
   auto kernel = pkv::paged_decode_kernel<C, T, D>;
   const size_t smem = pkv::DecodeSmem<C>::kBytes;
-  int rc = ensure_smem(kernel, smem);
+  static std::atomic<uint64_t> smem_set{0};
+  int rc = ensure_smem(kernel, smem, smem_set);
   if (rc != PKV_OK) return rc;
   dim3 grid((unsigned)p.Hkv, (unsigned)p.max_parts, (unsigned)B);
   kernel<<<grid, pkv::kWarps * 32, smem, stream>>>(p, mk, mv);

@@ -170,6 +170,9 @@ def test_device_error_flags_and_safety():
     assert pkv.device_errors() == pkv.DEVERR_SLOT
     assert torch.equal(raw(before), raw(dev["k_cache"]))
 
+    # a table entry outside the pool: flagged, read as zeros, outputs stay finite
+    pkv.paged_kv_write(dev["k_new"], dev["v_new"], dev["k_cache"], dev["v_cache"],
+                       dev["slot_mapping"])
     bt = dev["block_tables"].clone()
     bt[0, 0] = wl.num_blocks + 3
     out = torch.empty_like(dev["q"])
