@@ -340,7 +340,7 @@ def run_ours(args, rank, world, local_rank):
     dec_avg_ms = statistics.fmean(dec_ms)
     achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
     G = wl.G
-    tc = wl.dtype == "bf16" and (args.path == "tensor_cores" or (args.path == "auto" and G >= 3))
+    tc = wl.dtype == "bf16" and (args.path != "cuda_cores" or G > 8)
     kernel = "paged_decode_kernel<MmaConsumer>" if tc else "paged_decode_kernel<SimtConsumer>"
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),

@@ -188,7 +188,7 @@ int pkv_device_errors(uint32_t *bits, int clear);
 /*
  * Arithmetic units used by paged_attention_decode, set for the whole process
  * (for testing and measuring both kernels):
- *   PKV_PATH_AUTO          bf16 with G >= 3 on tensor cores, all else on CUDA cores;
+ *   PKV_PATH_AUTO          every bf16 call on tensor cores, fp32 on CUDA cores;
  *   PKV_PATH_CUDA_CORES    fp32 FMAs whenever G <= 8;
  *   PKV_PATH_TENSOR_CORES  warp-level bf16 MMA for every bf16 call.
  * fp32 always runs on CUDA cores.  Returns the previous mode, or

@@ -18,10 +18,10 @@
 //  * online softmax in fp32 (running max and sum, exp2 with the scale folded
 //    into log2 units), per warp; warps and then partitions are merged with a
 //    log-sum-exp rescale;
-//  * grouped heads (G > 2, bf16) run the score and PV products on the tensor
-//    cores with a warp-level m16n8k16 MMA: tokens are M, the G heads are N
+//  * bf16 runs the score and PV products on the tensor cores with a
+//    warp-level m16n8k16 MMA: tokens are M, the G heads of a KV head are N
 //    (padded to 8), D is K; PV computes O^T = V^T P^T with P transposed in
-//    registers by movmatrix.  Smaller G and fp32 use CUDA-core FMAs;
+//    registers by movmatrix.  fp32 (and, on request, bf16) uses CUDA-core FMAs;
 //  * a sequence split into several partitions writes partial (max, sum,
 //    weighted V) to the workspace; the CTA that finishes last for a
 //    (b, kvh) -- found with an atomic ticket, no spinning -- merges them.
