@@ -57,7 +57,9 @@ enum {
     PKV_ERR_OUT_OF_RANGE = -2, /* a host-checkable size or bound is out of range */
     PKV_ERR_WORKSPACE = -3,    /* decode workspace missing or too small */
     PKV_ERR_CUDA = -4,         /* a CUDA call failed; see pkv_last_cuda_error() */
-    PKV_ERR_UNSUPPORTED = -5   /* valid but unsupported shape (head dim, block size, G) */
+    PKV_ERR_UNSUPPORTED = -5,  /* valid but unsupported shape (head dim, block size, G) */
+    PKV_ERR_SCRATCH_LIMIT = -6 /* paged_attention_decode_noalloc: sizes need more than
+                                  PKV_NOALLOC_SCRATCH_BYTES of scratch */
 };
 
 /* Device error bits (pkv_device_errors). */
@@ -152,6 +154,39 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
                            int64_t num_blocks, float scale, pkv_dtype dtype,
                            int partition_size, void *workspace, size_t workspace_bytes,
                            pkv_stream_t stream);
+
+/*
+ * paged_attention_decode_noalloc: the same decode as paged_attention_decode
+ * for callers that cannot allocate device memory and have no workspace of
+ * their own to lend.  Examples are a host program whose device memory is
+ * entirely owned by its own pool allocator, and a serving loop that must not
+ * call cudaMalloc mid-step because the call may synchronise the device.  The
+ * pages describe no such entry point; it has no counterpart there.
+ *
+ * Arguments and results are those of paged_attention_decode without the
+ * workspace.  The split-partition scratch lives in one array of
+ * PKV_NOALLOC_SCRATCH_BYTES in the library's device memory.  Every GPU that
+ * loads the library holds that array until the process exits.  The call
+ * allocates and frees nothing.
+ *   - Sizes whose scratch (paged_attention_decode_workspace_size) exceeds
+ *     PKV_NOALLOC_SCRATCH_BYTES are rejected with PKV_ERR_SCRATCH_LIMIT before
+ *     anything is enqueued.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current.  Make that first call
+ *     before any stream capture.
+ *   - All calls share the one array, and it keeps what the last call left.
+ *     Each call therefore clears the part that must start at zero (the
+ *     partition counters) on `stream` before the decode.  Calls that overlap
+ *     on the GPU (other streams, other host threads) race on the array and
+ *     give wrong results; serialise them.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+int paged_attention_decode_noalloc(void *out, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_tables,
+                                   int max_blocks, const int32_t *seq_lens, int max_seq_len, int B,
+                                   int Hq, int Hkv, int D, int block_size, int64_t num_blocks,
+                                   float scale, pkv_dtype dtype, int partition_size,
+                                   pkv_stream_t stream);
 
 /*
  * copy_blocks: block-granularity copy-on-write copies.  Physical blocks are

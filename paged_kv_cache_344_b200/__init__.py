@@ -35,6 +35,8 @@ DEVERR_SEQLEN = 0x2
 DEVERR_BLOCK_ID = 0x4
 DEVERR_COPY = 0x8
 DEVERR_TIMEOUT = 0x10
+PKV_ERR_SCRATCH_LIMIT = -6
+NOALLOC_SCRATCH_BYTES = 16 << 20  # PKV_NOALLOC_SCRATCH_BYTES
 
 _lib = None
 
@@ -73,6 +75,9 @@ def lib() -> ctypes.CDLL:
     L.paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
                                          i32, i64, f32, i32, i32, vp, sz, vp]
     L.paged_attention_decode.restype = i32
+    L.paged_attention_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
+                                                 i32, i32, i32, i64, f32, i32, i32, vp]
+    L.paged_attention_decode_noalloc.restype = i32
     L.copy_blocks.argtypes = [vp, vp, vp, i64, i64, i64, vp]
     L.copy_blocks.restype = i32
     L.pkv_status_string.argtypes = [i32]
@@ -153,6 +158,19 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, max
         block_tables.shape[1], _ptr(seq_lens), int(max_seq_len), B, Hq, Hkv, D, bs, NB,
         float(scale), _dtype_code(q), int(partition_size), _ptr(workspace), ws_bytes,
         _stream(q, stream)))
+
+
+def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, max_seq_len,
+                                   scale, partition_size=0, stream=None) -> None:
+    """The decode without a workspace argument, for callers that cannot allocate device
+    memory: its split-partition scratch is a fixed array inside the library (see
+    ``include/pagedkv.h``).  Calls that overlap on the GPU race on that array."""
+    B, Hq, D = q.shape
+    NB, bs, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    _check("paged_attention_decode_noalloc", lib().paged_attention_decode_noalloc(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), int(max_seq_len), B, Hq, Hkv, D, bs, NB,
+        float(scale), _dtype_code(q), int(partition_size), _stream(q, stream)))
 
 
 def copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:

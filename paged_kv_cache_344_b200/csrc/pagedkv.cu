@@ -309,6 +309,63 @@ int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int6
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free decode.  Its scratch is this file-scope device array.  In
+// host code the symbol is only a stand-in for the array; the device address
+// comes from cudaGetSymbolAddress, looked up once per device.
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+int noalloc_scratch(void** ptr) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= 64) return PKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_tables,
+                                   int max_blocks, const int32_t* seq_lens, int max_seq_len, int B,
+                                   int Hq, int Hkv, int D, int block_size, int64_t num_blocks,
+                                   float scale, pkv_dtype dtype, int partition_size,
+                                   pkv_stream_t stream) {
+  DecodeShape shape;
+  int rc = decode_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape);
+  if (rc != PKV_OK) return rc;
+  if (shape.bytes > (size_t)PKV_NOALLOC_SCRATCH_BYTES) return PKV_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if (shape.bytes > 0) {
+    if ((rc = noalloc_scratch(&scratch)) != PKV_OK) return rc;
+    // The partition counters must start at zero; the array keeps whatever the
+    // previous call left, so clear them on this call's stream first.
+    cudaError_t e = cudaMemsetAsync(scratch, 0, shape.off_ml, stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return paged_attention_decode(out, q, k_cache, v_cache, block_tables, max_blocks, seq_lens,
+                                max_seq_len, B, Hq, Hkv, D, block_size, num_blocks, scale, dtype,
+                                partition_size, scratch, shape.bytes > 0 ? PKV_NOALLOC_SCRATCH_BYTES : 0,
+                                stream);
+}
+
 const char* pkv_status_string(int status) {
   switch (status) {
     case PKV_OK: return "ok";
@@ -317,6 +374,7 @@ const char* pkv_status_string(int status) {
     case PKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case PKV_ERR_CUDA: return "CUDA error (see pkv_last_cuda_error)";
     case PKV_ERR_UNSUPPORTED: return "unsupported shape";
+    case PKV_ERR_SCRATCH_LIMIT: return "sizes need more scratch than the allocation-free decode has";
     default: return "unknown status";
   }
 }
