@@ -211,6 +211,7 @@ def run_ours(args, rank, world, local_rank):
     dev_name = f"cuda:{local_rank}"
     pkv.set_decode_path({"auto": pkv.PKV_PATH_AUTO, "cuda_cores": pkv.PKV_PATH_CUDA_CORES,
                          "tensor_cores": pkv.PKV_PATH_TENSOR_CORES}[args.path])
+    pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED if args.split == "balanced" else pkv.PKV_SPLIT_FIXED)
     wl = workloads.make(args.config)
     dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
     meta = {
@@ -341,7 +342,8 @@ def run_ours(args, rank, world, local_rank):
     achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
     G = wl.G
     tc = wl.dtype == "bf16" and (args.path != "cuda_cores" or G > 8)
-    kernel = "paged_decode_kernel<MmaConsumer>" if tc else "paged_decode_kernel<SimtConsumer>"
+    kernel = ("paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
+        + ("<MmaConsumer>" if tc else "<SimtConsumer>")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
                 "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
@@ -374,7 +376,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
                           else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "decode_path": args.path, "partition_tokens": part},
+                   "decode_path": args.path, "decode_split": args.split,
+                   "partition_tokens": part},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -431,6 +434,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=["auto", "cuda_cores", "tensor_cores"], default="auto",
                     help="decode kernel family (library default: auto)")
+    ap.add_argument("--split", choices=["fixed", "balanced"], default="fixed",
+                    help="decode work split (library default: fixed-length partitions)")
     ap.add_argument("--partition", type=int, default=0,
                     help="decode partition length in tokens (0 = library choice)")
     args = ap.parse_args()

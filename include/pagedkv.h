@@ -91,17 +91,19 @@ int paged_kv_write(const void *k, const void *v, void *k_cache, void *v_cache,
 
 /*
  * Partition length (tokens) that paged_attention_decode uses for these sizes:
- * `partition_size` itself when it is > 0, otherwise the library's choice.
- * The choice is a multiple of 16 and depends only on the arguments.
- * Returns a negative status for invalid arguments.
+ * `partition_size` itself when it is > 0, otherwise the library's choice, a
+ * multiple of 16 that depends only on the arguments (0 when the process runs
+ * the work-balanced split, see pkv_set_decode_split).  Returns a negative
+ * status for invalid arguments.
  */
 int paged_attention_decode_partition_size(int B, int Hkv, int max_seq_len, int block_size,
                                           int partition_size);
 
 /*
- * Workspace bytes paged_attention_decode needs for these sizes: 0 when every
- * sequence fits in one partition.  It is a pure host function with no CUDA
- * calls.  Returns 0 for invalid arguments (the call then reports the error).
+ * Workspace bytes paged_attention_decode needs for these sizes, in either
+ * split mode (0 when no partial results can arise).  It is a pure host function
+ * with no CUDA calls.  Returns 0 for invalid arguments (the call then reports
+ * the error).
  */
 size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_seq_len,
                                              int block_size, int partition_size);
@@ -124,10 +126,12 @@ size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int 
  * exactly and the result is rounded to nearest even.  Slots past L in the
  * last block, and table entries past ceil(L / block_size), are never read.
  *
- * Long sequences are split into partitions of P tokens
- * (paged_attention_decode_partition_size).  Each partition yields a partial
- * (max, sum, weighted V), and the partials are merged with a log-sum-exp
- * rescale in the same launch.
+ * Work split.  Each sequence is cut into partitions of P tokens (P =
+ * partition_size, or the library's choice when it is 0), one CTA per (KV
+ * head, partition, sequence).  pkv_set_decode_split selects a work-balanced
+ * persistent split instead.  A (sequence, KV head) cut in several pieces yields
+ * one partial (max, sum, weighted V) per piece.  The partials are merged with a
+ * log-sum-exp rescale in the same launch.
  *
  *   out             device [B][Hq][D], written
  *   q               device [B][Hq][D]
@@ -231,6 +235,29 @@ int pkv_device_errors(uint32_t *bits, int clear);
  */
 enum { PKV_PATH_AUTO = 0, PKV_PATH_CUDA_CORES = 1, PKV_PATH_TENSOR_CORES = 2 };
 int pkv_set_decode_path(int mode);
+
+/*
+ * How paged_attention_decode with partition_size == 0 cuts the work, set for
+ * the whole process:
+ *   PKV_SPLIT_FIXED (default)  partitions of a library-chosen length, one CTA
+ *                              each (grid over KV heads, partitions, sequences);
+ *   PKV_SPLIT_BALANCED         a persistent grid in which every warp takes an
+ *                              equal contiguous range of one KV head's stream of
+ *                              16-token stages (B <= 2048; otherwise FIXED).
+ * Both give results within the same bounds.  paged_attention_decode_workspace_size
+ * covers either mode.  Returns the previous mode, or PKV_ERR_INVALID_ARG.
+ */
+enum { PKV_SPLIT_FIXED = 0, PKV_SPLIT_BALANCED = 1 };
+int pkv_set_decode_split(int mode);
+
+/*
+ * Number of CTAs of the work-balanced decode kernel, set for the whole process
+ * (for tests and measurements): 0 (default) launches as many as are resident
+ * at once, at most 2 per SM; n > 0 launches min(n, 296).  Results satisfy the
+ * same bounds for every value.  Returns the previous value, or
+ * PKV_ERR_INVALID_ARG for n < 0.
+ */
+int pkv_set_decode_ctas(int ctas);
 
 #ifdef __cplusplus
 }

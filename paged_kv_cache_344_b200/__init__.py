@@ -36,6 +36,8 @@ DEVERR_BLOCK_ID = 0x4
 DEVERR_COPY = 0x8
 DEVERR_TIMEOUT = 0x10
 PKV_ERR_SCRATCH_LIMIT = -6
+PKV_SPLIT_FIXED = 0
+PKV_SPLIT_BALANCED = 1
 NOALLOC_SCRATCH_BYTES = 16 << 20  # PKV_NOALLOC_SCRATCH_BYTES
 
 _lib = None
@@ -87,6 +89,10 @@ def lib() -> ctypes.CDLL:
     L.pkv_device_errors.restype = i32
     L.pkv_set_decode_path.argtypes = [i32]
     L.pkv_set_decode_path.restype = i32
+    L.pkv_set_decode_split.argtypes = [i32]
+    L.pkv_set_decode_split.restype = i32
+    L.pkv_set_decode_ctas.argtypes = [i32]
+    L.pkv_set_decode_ctas.restype = i32
     _lib = L
     return L
 
@@ -193,4 +199,18 @@ def set_decode_path(mode: int) -> int:
     """Select CUDA-core / tensor-core decode kernels process-wide; returns the old mode."""
     r = lib().pkv_set_decode_path(int(mode))
     _check("pkv_set_decode_path", min(r, 0))
+    return r
+
+
+def set_decode_ctas(ctas: int) -> int:
+    """CTA count of the work-balanced decode (0 = as many as are resident); returns the old."""
+    r = lib().pkv_set_decode_ctas(int(ctas))
+    _check("pkv_set_decode_ctas", min(r, 0))
+    return r
+
+
+def set_decode_split(mode: int) -> int:
+    """Fixed-length partitions (default) or the work-balanced split; returns the old mode."""
+    r = lib().pkv_set_decode_split(int(mode))
+    _check("pkv_set_decode_split", min(r, 0))
     return r

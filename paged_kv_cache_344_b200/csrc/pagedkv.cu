@@ -11,12 +11,15 @@
 #include <cmath>
 #include <mutex>
 
+#include "pkv_decode_balanced.cuh"
 #include "pkv_write_copy.cuh"
 
 namespace {
 
 thread_local int g_last_cuda_error = 0;
 std::atomic<int> g_decode_path{PKV_PATH_AUTO};
+std::atomic<int> g_decode_ctas{0};  // 0: as many as fit (at most 2 per SM)
+std::atomic<int> g_decode_split{PKV_SPLIT_FIXED};
 
 constexpr int kSmCount = 148;  // B200
 
@@ -86,23 +89,29 @@ int ensure_smem(Kernel kernel, size_t bytes, std::atomic<uint64_t>& done) {
 }
 
 int auto_partition(int B, int Hkv, int max_seq_len) {
-  // Long partitions: every CTA pays a start-up (table ids, q, pipeline fill)
-  // and every extra partition a partial write and merge, and CTAs whose
-  // partition lies past a short sequence's end still occupy a slot briefly.
-  // Shorten them only until there are about three waves of CTAs
-  // (2 resident per SM).  Measured on B200: 4096 beats 2048, 1024 and 512 on
-  // the MHA, GQA and long-context workloads.
+  // About half the longest sequence, between 512 and 4096 tokens: the longest
+  // sequences are cut in two (halving the largest CTAs, which set the tail)
+  // while most sequences stay whole.  Longer partitions waste less on
+  // start-up and on partial results; every partition costs a CTA start-up
+  // (table ids, q, pipeline fill) and a partial write and merge.  Then shorten
+  // until there are about three waves of CTAs (3 resident per SM).  Measured on
+  // B200: MHA (max 2049) best at 1024, GQA (max 4097) at 2048, long context
+  // (max 131073) at 4096.
   const int64_t units = (int64_t)B * Hkv;
-  const int64_t target = (int64_t)kSmCount * 2 * 3;
-  int P = 4096;
-  while (P > 512 && units * ceil_div(max_seq_len > 0 ? max_seq_len : 1, P) < target) P /= 2;
+  const int64_t target = (int64_t)kSmCount * 3 * 3;
+  const int64_t L = max_seq_len > 0 ? max_seq_len : 1;
+  int P = 512;
+  while (P < 4096 && (int64_t)P * 2 <= L / 2) P *= 2;
+  while (P > 512 && units * ceil_div(L, P) < target) P /= 2;
   return P;
 }
 
 struct DecodeShape {
-  int P;
+  bool balanced;  // work-balanced persistent kernel (else fixed-length partitions)
+  int P;          // partition length of the fixed split (0 when balanced)
   int max_parts;
-  size_t off_ml, off_acc, bytes;
+  size_t off_ml, off_acc, bytes;  // workspace layout and size of the split in use
+  size_t ws_bytes;                // size reported to callers: covers either split
 };
 
 int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
@@ -111,21 +120,38 @@ int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
     return PKV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
   if (partition_size < 0 || partition_size % pkv::kStageTokens != 0) return PKV_ERR_INVALID_ARG;
-  const int P = partition_size > 0 ? partition_size : auto_partition(B, Hkv, max_seq_len);
-  const int64_t mp = max_seq_len > 0 ? ceil_div(max_seq_len, P) : 1;
-  if (mp > 65535) return PKV_ERR_OUT_OF_RANGE;
-  s->P = P;
-  s->max_parts = (int)mp;
-  if (mp <= 1 || B == 0) {
-    s->off_ml = s->off_acc = s->bytes = 0;
-    return PKV_OK;
-  }
   const size_t G = (size_t)(Hq / Hkv);
   const size_t units = (size_t)B * Hkv;
   auto align256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
-  s->off_ml = align256(units * sizeof(uint32_t));
-  s->off_acc = s->off_ml + align256(units * mp * G * sizeof(float2));
-  s->bytes = s->off_acc + units * mp * G * (size_t)D * sizeof(float);
+
+  // Fixed-length partitions (the default split).
+  const int P = partition_size > 0 ? partition_size : auto_partition(B, Hkv, max_seq_len);
+  const int64_t mp = max_seq_len > 0 ? ceil_div(max_seq_len, P) : 1;
+  if (mp > 65535) return PKV_ERR_OUT_OF_RANGE;
+  size_t f_ml = 0, f_acc = 0, f_bytes = 0;
+  if (mp > 1 && B > 0) {
+    f_ml = align256(units * sizeof(uint32_t));
+    f_acc = f_ml + align256(units * mp * G * sizeof(float2));
+    f_bytes = f_acc + units * mp * G * (size_t)D * sizeof(float);
+  }
+  // Work-balanced split (opt-in): needs the per-sequence prefix in shared memory
+  // and a stage count that fits in 31 bits.
+  const int64_t max_stages = (int64_t)B * Hkv * ceil_div(max_seq_len, pkv::kStageTokens);
+  const bool bal_ok = partition_size == 0 && B <= pkv::kBalancedMaxB && max_stages < 0x7fffffffLL;
+  size_t b_ml = 0, b_acc = 0, b_bytes = 0;
+  if (bal_ok && B > 0) {
+    const size_t slots = pkv::balanced_slots((size_t)B, (size_t)Hkv);
+    b_ml = align256(units * sizeof(uint32_t));
+    b_acc = b_ml + align256(slots * G * sizeof(float2));
+    b_bytes = b_acc + slots * G * (size_t)D * sizeof(float);
+  }
+  s->balanced = bal_ok && g_decode_split.load(std::memory_order_relaxed) == PKV_SPLIT_BALANCED;
+  s->P = s->balanced ? 0 : P;
+  s->max_parts = s->balanced ? 0 : (int)mp;
+  s->off_ml = s->balanced ? b_ml : f_ml;
+  s->off_acc = s->balanced ? b_acc : f_acc;
+  s->bytes = s->balanced ? b_bytes : f_bytes;
+  s->ws_bytes = std::max(f_bytes, b_bytes);
   return PKV_OK;
 }
 
@@ -143,23 +169,58 @@ int launch_decode(const pkv::DecodeParams& p, int B, const CUtensorMap& mk, cons
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
+// Balanced kernel: a persistent grid of as many CTAs as are resident at once
+// (at most 2 per SM), so that every worker starts at the same time.
+template <class C, typename T, int D>
+int launch_balanced(const pkv::DecodeParams& p, const CUtensorMap& mk, const CUtensorMap& mv,
+                    cudaStream_t stream) {
+  auto kernel = pkv::paged_decode_balanced_kernel<C, T, D>;
+  static std::atomic<uint64_t> smem_set{0};
+  static std::atomic<int> resident[64];
+  int rc = ensure_smem(kernel, pkv::BalancedSmem<C>::bytes(pkv::kBalancedMaxB), smem_set);
+  if (rc != PKV_OK) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  int ctas = resident[dev & 63].load(std::memory_order_relaxed);
+  if (ctas == 0) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &per_sm, kernel, pkv::kWarps * 32, pkv::BalancedSmem<C>::bytes(pkv::kBalancedMaxB));
+    if (e != cudaSuccess) return cuda_fail(e);
+    ctas = std::max(1, std::min(sms * std::min(per_sm, 2), pkv::kBalancedMaxCtas));
+    resident[dev & 63].store(ctas, std::memory_order_relaxed);
+  }
+  const int forced = g_decode_ctas.load(std::memory_order_relaxed);
+  if (forced > 0) ctas = std::min(forced, pkv::kBalancedMaxCtas);
+  kernel<<<ctas, pkv::kWarps * 32, pkv::BalancedSmem<C>::bytes(p.B), stream>>>(p, mk, mv);
+  e = cudaGetLastError();
+  return e == cudaSuccess ? PKV_OK : cuda_fail(e);
+}
+
+template <class C, typename T, int D>
+int launch_any(const pkv::DecodeParams& p, bool balanced, const CUtensorMap& mk,
+               const CUtensorMap& mv, cudaStream_t s) {
+  return balanced ? launch_balanced<C, T, D>(p, mk, mv, s) : launch_decode<C, T, D>(p, p.B, mk, mv, s);
+}
+
 template <typename T, int D>
-int dispatch_simt(const pkv::DecodeParams& p, int B, const CUtensorMap& mk,
+int dispatch_simt(const pkv::DecodeParams& p, bool bal, const CUtensorMap& mk,
                   const CUtensorMap& mv, cudaStream_t s) {
-  if (p.G == 1) return launch_decode<pkv::SimtConsumer<T, D, 1>, T, D>(p, B, mk, mv, s);
-  if (p.G == 2) return launch_decode<pkv::SimtConsumer<T, D, 2>, T, D>(p, B, mk, mv, s);
-  if (p.G <= 4) return launch_decode<pkv::SimtConsumer<T, D, 4>, T, D>(p, B, mk, mv, s);
-  if (p.G <= 8) return launch_decode<pkv::SimtConsumer<T, D, 8>, T, D>(p, B, mk, mv, s);
+  if (p.G == 1) return launch_any<pkv::SimtConsumer<T, D, 1>, T, D>(p, bal, mk, mv, s);
+  if (p.G == 2) return launch_any<pkv::SimtConsumer<T, D, 2>, T, D>(p, bal, mk, mv, s);
+  if (p.G <= 4) return launch_any<pkv::SimtConsumer<T, D, 4>, T, D>(p, bal, mk, mv, s);
+  if (p.G <= 8) return launch_any<pkv::SimtConsumer<T, D, 8>, T, D>(p, bal, mk, mv, s);
   return PKV_ERR_UNSUPPORTED;
 }
 
 template <int D>
-int dispatch_mma(const pkv::DecodeParams& p, int B, const CUtensorMap& mk, const CUtensorMap& mv,
-                 cudaStream_t s) {
-  if (p.G <= 8)
-    return launch_decode<pkv::MmaConsumer<D, 1>, __nv_bfloat16, D>(p, B, mk, mv, s);
-  if (p.G <= 16)
-    return launch_decode<pkv::MmaConsumer<D, 2>, __nv_bfloat16, D>(p, B, mk, mv, s);
+int dispatch_mma(const pkv::DecodeParams& p, bool bal, const CUtensorMap& mk,
+                 const CUtensorMap& mv, cudaStream_t s) {
+  if (p.G <= 8) return launch_any<pkv::MmaConsumer<D, 1>, __nv_bfloat16, D>(p, bal, mk, mv, s);
+  if (p.G <= 16) return launch_any<pkv::MmaConsumer<D, 2>, __nv_bfloat16, D>(p, bal, mk, mv, s);
   return PKV_ERR_UNSUPPORTED;
 }
 
@@ -215,7 +276,7 @@ size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int 
                                              int block_size, int partition_size) {
   DecodeShape s;
   if (decode_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &s) != PKV_OK) return 0;
-  return s.bytes;
+  return s.ws_bytes;
 }
 
 int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
@@ -257,6 +318,7 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
   p.ws_count = shape.bytes ? reinterpret_cast<uint32_t*>(ws) : nullptr;
   p.ws_ml = shape.bytes ? reinterpret_cast<float2*>(ws + shape.off_ml) : nullptr;
   p.ws_acc = shape.bytes ? reinterpret_cast<float*>(ws + shape.off_acc) : nullptr;
+  p.B = B;
   p.max_blocks = max_blocks;
   p.max_seq_len = max_seq_len;
   p.Hq = Hq;
@@ -274,18 +336,19 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
   if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, tc)) != PKV_OK) return rc;
   if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, tc)) != PKV_OK) return rc;
 
+  const bool bal = shape.balanced;
   if (tc) {
-    if (D == 64) return dispatch_mma<64>(p, B, mk, mv, stream);
-    if (D == 128) return dispatch_mma<128>(p, B, mk, mv, stream);
-    return dispatch_mma<256>(p, B, mk, mv, stream);
+    if (D == 64) return dispatch_mma<64>(p, bal, mk, mv, stream);
+    if (D == 128) return dispatch_mma<128>(p, bal, mk, mv, stream);
+    return dispatch_mma<256>(p, bal, mk, mv, stream);
   }
   if (dtype == PKV_BF16) {
-    if (D == 64) return dispatch_simt<__nv_bfloat16, 64>(p, B, mk, mv, stream);
-    if (D == 128) return dispatch_simt<__nv_bfloat16, 128>(p, B, mk, mv, stream);
-    return dispatch_simt<__nv_bfloat16, 256>(p, B, mk, mv, stream);
+    if (D == 64) return dispatch_simt<__nv_bfloat16, 64>(p, bal, mk, mv, stream);
+    if (D == 128) return dispatch_simt<__nv_bfloat16, 128>(p, bal, mk, mv, stream);
+    return dispatch_simt<__nv_bfloat16, 256>(p, bal, mk, mv, stream);
   }
-  if (D == 64) return dispatch_simt<float, 64>(p, B, mk, mv, stream);
-  return dispatch_simt<float, 128>(p, B, mk, mv, stream);
+  if (D == 64) return dispatch_simt<float, 64>(p, bal, mk, mv, stream);
+  return dispatch_simt<float, 128>(p, bal, mk, mv, stream);
 }
 
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int64_t P,
@@ -391,6 +454,16 @@ int pkv_device_errors(uint32_t* bits, int clear) {
     if (e != cudaSuccess) return cuda_fail(e);
   }
   return PKV_OK;
+}
+
+int pkv_set_decode_split(int mode) {
+  if (mode != PKV_SPLIT_FIXED && mode != PKV_SPLIT_BALANCED) return PKV_ERR_INVALID_ARG;
+  return g_decode_split.exchange(mode);
+}
+
+int pkv_set_decode_ctas(int ctas) {
+  if (ctas < 0) return PKV_ERR_INVALID_ARG;
+  return g_decode_ctas.exchange(ctas);
 }
 
 int pkv_set_decode_path(int mode) {

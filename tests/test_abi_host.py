@@ -41,16 +41,29 @@ def test_status_strings(lib):
 
 
 def test_partition_and_workspace_sizes(lib):
-    # requested partition sizes are honoured; the automatic one is a multiple of 16
+    # requested partition sizes are honoured; the automatic one is a multiple of 16, or 0
+    # while the process runs the work-balanced split
     assert pkv.paged_attention_decode_partition_size(8, 8, 131073, 16, 512) == 512
-    for B, Hkv, L in [(64, 40, 2049), (256, 8, 4097), (8, 8, 131073), (128, 8, 1281), (4, 4, 34)]:
+    for B, Hkv, L in [(64, 40, 2049), (256, 8, 4097), (8, 8, 131073), (128, 8, 1281), (4, 4, 34),
+                      (4096, 8, 2049)]:
         P = pkv.paged_attention_decode_partition_size(B, Hkv, L, 16, 0)
         assert P > 0 and P % 16 == 0
+    old = pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED)
+    try:
+        assert pkv.paged_attention_decode_partition_size(64, 40, 2049, 16, 0) == 0
+        assert pkv.paged_attention_decode_partition_size(4096, 8, 2049, 16, 0) > 0  # B > 2048
+    finally:
+        pkv.set_decode_split(old)
     with pytest.raises(pkv.PagedKVError):
         pkv.paged_attention_decode_partition_size(8, 8, 100, 16, 24)  # not a multiple of 16
-    # a single partition needs no workspace
-    assert pkv.paged_attention_decode_workspace_size(4, 4, 4, 64, 34, 16, 0) == 0
+    # fixed-length partitions: one partition needs no workspace
     assert pkv.paged_attention_decode_workspace_size(8, 64, 8, 128, 1000, 16, 1024) == 0
+    # the size covers the balanced split too: counters + one partial slot per unit and per
+    # worker (1184 workers)
+    slots = 4 * 4 + 1184
+    ws = pkv.paged_attention_decode_workspace_size(4, 4, 4, 64, 34, 16, 0)
+    assert slots * (64 + 2) * 4 <= ws <= slots * (64 + 2) * 4 + 1024
+    assert pkv.paged_attention_decode_workspace_size(0, 4, 4, 64, 34, 16, 0) == 0
     # split partitions: counters + (max, sum) + D floats per (b, kvh, part, head)
     ws = pkv.paged_attention_decode_workspace_size(8, 64, 8, 128, 131073, 16, 2048)
     parts = -(-131073 // 2048)
@@ -112,6 +125,20 @@ def test_write_and_copy_reject_bad_arguments(lib):
     assert c(P=-1) == ERR_ARG
     assert c(nb=0) == ERR_ARG
     assert c(P=0) == 0
+
+
+def test_decode_split_selector(lib):
+    old = pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED)
+    assert pkv.set_decode_split(old) == pkv.PKV_SPLIT_BALANCED
+    with pytest.raises(pkv.PagedKVError):
+        pkv.set_decode_split(5)
+
+
+def test_decode_cta_selector(lib):
+    old = pkv.set_decode_ctas(7)
+    assert pkv.set_decode_ctas(old) == 7
+    with pytest.raises(pkv.PagedKVError):
+        pkv.set_decode_ctas(-1)
 
 
 def test_decode_path_selector(lib):

@@ -84,6 +84,27 @@ def test_partition_invariance(P, path):
     assert_attention_close(widen(out), ref, wl.dtype, f"P={P}")
 
 
+@pytest.mark.parametrize("ctas", [1, 3, 37, 296])
+@pytest.mark.parametrize("name,sd", [("mha", 8), ("gqa16", 8), ("long", 16), ("share_fork", 4),
+                                     ("tiny", 1)])
+def test_balanced_split_any_worker_count(name, sd, ctas):
+    """The work-balanced kernel cuts the stage stream into one range per warp; with 1 to
+    296 CTAs units are cut into every pattern of pieces (inside one worker, across two,
+    across many, one stage per worker) and must still give the oracle's result."""
+    old = pkv.set_decode_ctas(ctas)
+    old_split = pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED)
+    try:
+        wl, host = _case(name, sd)
+        dev = device_inputs(wl, host)
+        out = gpu_step(wl, dev)
+        _, _, ref = oracle_step(wl, host)
+        assert_attention_close(widen(out), ref, wl.dtype, f"{name} ctas={ctas}")
+        assert pkv.device_errors() == 0
+    finally:
+        pkv.set_decode_ctas(old)
+        pkv.set_decode_split(old_split)
+
+
 def test_workspace_reuse_and_streams():
     """Two calls on one workspace (its counters must come back to zero) and a call on a
     side stream give identical results."""
