@@ -65,24 +65,27 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the device-code sources (the .cuh files holding the kernels)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_344_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        if name.endswith(".cuh"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(config: str):
+def recorded_traffic(config: str, partition: int):
     """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
-    current kernel sources (else None)."""
+    current kernel sources with the same partition length (else None)."""
     path = os.path.join(ROOT, "profiles", f"decode_{config}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     s = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
-    if not m or not s or s.group(1) != kernel_source_sha():
+    q = re.search(r"partition_tokens:\s*([0-9]+)", text)
+    if not m or not s or not q or s.group(1) != kernel_source_sha() or int(q.group(1)) != partition:
         return None
     return float(m.group(1))
 
@@ -345,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
     kernel = ("paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
         + ("<MmaConsumer>" if tc else "<SimtConsumer>")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config),
+                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config, part),
                 "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                 "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
                 "decode_us": round(dec_avg_ms * 1e3, 2),

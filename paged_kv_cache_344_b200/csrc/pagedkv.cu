@@ -100,8 +100,8 @@ int auto_partition(int B, int Hkv, int max_seq_len) {
   const int64_t units = (int64_t)B * Hkv;
   const int64_t target = (int64_t)kSmCount * 3 * 3;
   const int64_t L = max_seq_len > 0 ? max_seq_len : 1;
-  int P = 512;
-  while (P < 4096 && (int64_t)P * 2 <= L / 2) P *= 2;
+  int P = 512;  // the power of two nearest (in log scale) to L / 2
+  while (P < 4096 && (double)L / 2 >= (double)P * 1.4142135623730951) P *= 2;
   while (P > 512 && units * ceil_div(L, P) < target) P /= 2;
   return P;
 }

@@ -578,8 +578,9 @@ __global__ void __launch_bounds__(kWarps * 32)
       win_base += 32;
       win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane) : -1;
     }
-    const int rel = k - win_base;
-    const int id = __shfl_sync(kFull, rel < 32 ? win0 : win1, rel & 31);
+    // After the rotation above, k - win_base < 32: read win0 only.  (Naming win1
+    // here would make the shuffle wait for the window load just issued.)
+    const int id = __shfl_sync(kFull, win0, k - win_base);
     if (lane == 0) {
       const int s = k % C::kStages;
       const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;

@@ -184,9 +184,10 @@ __global__ void __launch_bounds__(kWarps * 32)
         win_base += 32;
         locate(win_base + 32 + lane, id1, sub1);  // consumed 32 stages from now
       }
-      const int rel = k - win_base;
-      const int id = __shfl_sync(kFull, rel < 32 ? id0 : id1, rel & 31);
-      const int sub = __shfl_sync(kFull, rel < 32 ? sub0 : sub1, rel & 31);
+      // After the rotation above, k - win_base < 32: read window 0 only.  (Naming
+      // window 1 here would make the shuffle wait for the load just issued.)
+      const int id = __shfl_sync(kFull, id0, k - win_base);
+      const int sub = __shfl_sync(kFull, sub0, k - win_base);
       if (lane == 0) {
         int row;
         if (id < 0 || id >= p.num_blocks) {
