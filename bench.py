@@ -242,8 +242,17 @@ def run_ours(args, rank, world, local_rank):
         "slot_mapping": torch.from_numpy(wl.slot_mapping).to(dev_name),
         "cow_pairs": torch.from_numpy(wl.cow_pairs).to(dev_name),
     }
-    ws_bytes = pkv.paged_attention_decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D,
-                                                         wl.max_seq_len, wl.bs, args.partition)
+    use_shared = args.decode == "shared_prefix" or (args.decode == "auto"
+                                                    and args.config.startswith("share"))
+    if use_shared:
+        ws_bytes = pkv.paged_attention_decode_shared_prefix_workspace_size(
+            wl.B, wl.Hq, wl.Hkv, wl.D, wl.max_seq_len, wl.bs, args.partition)
+        meta["group_offsets"] = torch.from_numpy(wl.group_offsets).to(dev_name)
+        meta["prefix_lens"] = torch.from_numpy(wl.prefix_lens).to(dev_name)
+        max_group = int(np.diff(wl.group_offsets).max())
+    else:
+        ws_bytes = pkv.paged_attention_decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D,
+                                                             wl.max_seq_len, wl.bs, args.partition)
     part = pkv.paged_attention_decode_partition_size(wl.B, wl.Hkv, wl.max_seq_len, wl.bs,
                                                      args.partition)
     ws = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev_name)
@@ -262,9 +271,15 @@ def run_ours(args, rank, world, local_rank):
                            d_in["slot_mapping"])
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        pkv.paged_attention_decode(o, d_in["q"], d_in["k_cache"], d_in["v_cache"],
-                                   d_in["block_tables"], d_in["seq_lens"], wl.max_seq_len,
-                                   wl.scale, workspace=ws, partition_size=args.partition)
+        if use_shared:
+            pkv.paged_attention_decode_shared_prefix(
+                o, d_in["q"], d_in["k_cache"], d_in["v_cache"], d_in["block_tables"],
+                d_in["seq_lens"], wl.max_seq_len, wl.scale, d_in["group_offsets"],
+                d_in["prefix_lens"], max_group, workspace=ws, partition_size=args.partition)
+        else:
+            pkv.paged_attention_decode(o, d_in["q"], d_in["k_cache"], d_in["v_cache"],
+                                       d_in["block_tables"], d_in["seq_lens"], wl.max_seq_len,
+                                       wl.scale, workspace=ws, partition_size=args.partition)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
@@ -330,7 +345,8 @@ def run_ours(args, rank, world, local_rank):
     # step i's output run on a copy stream and overlap the computation of step i (two sets
     # of step buffers; the KV cache itself stays resident).
     in_keys = [k for k in ("q", "k_new", "v_new", "block_tables", "seq_lens", "slot_mapping",
-                           "cow_pairs") if k != "cow_pairs" or has_cow]
+                           "cow_pairs", "group_offsets", "prefix_lens")
+               if k in d_in and (k != "cow_pairs" or has_cow)]
     host_in = {k: d_in[k].cpu().pin_memory() for k in in_keys}
     bufs = [dict(d_in), dict(d_in)]
     for k in in_keys:
@@ -390,7 +406,8 @@ def run_ours(args, rank, world, local_rank):
     achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
     G = wl.G
     tc = wl.dtype == "bf16" and (args.path != "cuda_cores" or G > 8)
-    kernel = ("paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
+    kernel = ("paged_decode_shared_kernel" if use_shared else
+              "paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
         + ("<MmaConsumer>" if tc else "<SimtConsumer>")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config, part),
@@ -424,6 +441,8 @@ def run_ours(args, rank, world, local_rank):
                    "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
                           else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "decode_entry": "paged_attention_decode_shared_prefix" if use_shared
+                   else "paged_attention_decode",
                    "decode_path": args.path, "decode_split": args.split,
                    "partition_tokens": part},
         "roofline": roofline,
@@ -485,6 +504,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", choices=["auto", "cuda_cores", "tensor_cores"], default="auto",
                     help="decode kernel family (library default: auto)")
+    ap.add_argument("--decode", choices=["auto", "plain", "shared_prefix"], default="auto",
+                    help="decode entry point (auto: shared-prefix decode for the shared-prefix "
+                         "workloads, the plain decode otherwise)")
     ap.add_argument("--split", choices=["fixed", "balanced"], default="fixed",
                     help="decode work split (library default: fixed-length partitions)")
     ap.add_argument("--partition", type=int, default=0,

@@ -68,6 +68,8 @@ enum {
 #define PKV_DEVERR_BLOCK_ID 0x4u /* a block-table id outside [0, num_blocks) was read as zeros */
 #define PKV_DEVERR_COPY 0x8u     /* copy_blocks skipped a pair with an id outside [0, num_blocks) */
 #define PKV_DEVERR_TIMEOUT 0x10u /* a pipeline wait gave up after its time limit */
+#define PKV_DEVERR_PREFIX 0x20u  /* shared-prefix decode: a member's table entries differ from
+                                    the group's first member, or a sequence is in no group */
 
 /*
  * paged_kv_write: the cache update.  [Explained] "Step 2: Allocate Blocks
@@ -158,6 +160,47 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
                            int64_t num_blocks, float scale, pkv_dtype dtype,
                            int partition_size, void *workspace, size_t workspace_bytes,
                            pkv_stream_t stream);
+
+/*
+ * paged_attention_decode_shared_prefix: paged_attention_decode for batches in
+ * which consecutive sequences share the physical blocks of a prefix: decode
+ * branches of one request, parallel samples, a common prompt.  Physical blocks
+ * are shared through identical table entries ([Wiki] "How it works";
+ * [Index] "Complex Decoding (Beam Search & Parallel Sampling)").  The result
+ * is the same; each shared block is read once per group instead of once per
+ * member.  Prefix pieces score one read of the shared K/V against the queries
+ * of up to 16 / G members at once, stacked in the tensor-core N dimension.
+ * Pieces over each sequence's own tokens follow, as in paged_attention_decode.
+ * The pieces' partials are merged in the same launch.
+ *   group_offsets  device [n_groups + 1] int32: group g is sequences
+ *                  group_offsets[g] .. group_offsets[g+1]-1.  The offsets start
+ *                  at 0, end at B and never decrease (a group may have one member).
+ *   prefix_lens    device [n_groups] int32: leading tokens whose blocks are
+ *                  the same physical blocks in every member (equal table
+ *                  entries).  The decode uses min(prefix_len, shortest member's
+ *                  length), rounded down to a multiple of 16.  0 means nothing shared.
+ *   max_group_size host upper bound of the group sizes.
+ * The other arguments are as for paged_attention_decode.  bf16 only, G <= 16.
+ * The workspace (paged_attention_decode_shared_prefix_workspace_size) follows the
+ * same rules as paged_attention_decode's: zero-filled before first use, left
+ * ready for the next call, not shared by overlapping calls.  A prefix piece checks the
+ * members' table entries against the first member's; a mismatch, or a sequence
+ * that no group covers, flags PKV_DEVERR_PREFIX.
+ */
+int paged_attention_decode_shared_prefix(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         int max_blocks, const int32_t *seq_lens, int max_seq_len,
+                                         const int32_t *group_offsets, const int32_t *prefix_lens,
+                                         int n_groups, int max_group_size, int B, int Hq, int Hkv,
+                                         int D, int block_size, int64_t num_blocks, float scale,
+                                         pkv_dtype dtype, int partition_size, void *workspace,
+                                         size_t workspace_bytes, pkv_stream_t stream);
+
+/* Workspace bytes of paged_attention_decode_shared_prefix (pure host function;
+ * 0 for invalid arguments). */
+size_t paged_attention_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D,
+                                                           int max_seq_len, int block_size,
+                                                           int partition_size);
 
 /*
  * paged_attention_decode_noalloc: the same decode as paged_attention_decode

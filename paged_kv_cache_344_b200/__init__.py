@@ -35,6 +35,7 @@ DEVERR_SEQLEN = 0x2
 DEVERR_BLOCK_ID = 0x4
 DEVERR_COPY = 0x8
 DEVERR_TIMEOUT = 0x10
+DEVERR_PREFIX = 0x20
 PKV_ERR_SCRATCH_LIMIT = -6
 PKV_SPLIT_FIXED = 0
 PKV_SPLIT_BALANCED = 1
@@ -80,6 +81,12 @@ def lib() -> ctypes.CDLL:
     L.paged_attention_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
                                                  i32, i32, i32, i64, f32, i32, i32, vp]
     L.paged_attention_decode_noalloc.restype = i32
+    L.paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, vp, vp,
+                                                       i32, i32, i32, i32, i32, i32, i32, i64,
+                                                       f32, i32, i32, vp, sz, vp]
+    L.paged_attention_decode_shared_prefix.restype = i32
+    L.paged_attention_decode_shared_prefix_workspace_size.argtypes = [i32] * 7
+    L.paged_attention_decode_shared_prefix_workspace_size.restype = sz
     L.copy_blocks.argtypes = [vp, vp, vp, i64, i64, i64, vp]
     L.copy_blocks.restype = i32
     L.pkv_status_string.argtypes = [i32]
@@ -177,6 +184,30 @@ def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_l
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         block_tables.shape[1], _ptr(seq_lens), int(max_seq_len), B, Hq, Hkv, D, bs, NB,
         float(scale), _dtype_code(q), int(partition_size), _stream(q, stream)))
+
+
+def paged_attention_decode_shared_prefix_workspace_size(B, Hq, Hkv, D, max_seq_len, block_size,
+                                                        partition_size=0) -> int:
+    return int(lib().paged_attention_decode_shared_prefix_workspace_size(
+        B, Hq, Hkv, D, max_seq_len, block_size, partition_size))
+
+
+def paged_attention_decode_shared_prefix(out, q, k_cache, v_cache, block_tables, seq_lens,
+                                         max_seq_len, scale, group_offsets, prefix_lens,
+                                         max_group_size, workspace=None, partition_size=0,
+                                         stream=None) -> None:
+    """The decode for batches whose consecutive sequences share prefix blocks: group g is
+    sequences ``group_offsets[g] .. group_offsets[g+1]-1`` sharing ``prefix_lens[g]``
+    leading tokens; shared blocks are read once per group."""
+    B, Hq, D = q.shape
+    NB, bs, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("paged_attention_decode_shared_prefix", lib().paged_attention_decode_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(seq_lens), int(max_seq_len), _ptr(group_offsets),
+        _ptr(prefix_lens), prefix_lens.shape[0], int(max_group_size), B, Hq, Hkv, D, bs, NB,
+        float(scale), _dtype_code(q), int(partition_size), _ptr(workspace), ws_bytes,
+        _stream(q, stream)))
 
 
 def copy_blocks(k_cache, v_cache, block_mapping, stream=None) -> None:

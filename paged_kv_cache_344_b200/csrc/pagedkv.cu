@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "pkv_decode_balanced.cuh"
+#include "pkv_decode_shared.cuh"
 #include "pkv_write_copy.cuh"
 
 namespace {
@@ -235,6 +236,50 @@ bool use_tensor_cores(pkv_dtype dtype, int G) {
   return true;
 }
 
+// Shared-prefix decode: partition length, slots and workspace layout.
+struct SharedShape {
+  int P, max_pp, max_op, SL;
+  size_t off_ml, off_acc, bytes;
+};
+
+int shared_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
+                 int partition_size, SharedShape* s) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || max_seq_len < 0)
+    return PKV_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
+  if (partition_size < 0 || partition_size % pkv::kStageTokens != 0) return PKV_ERR_INVALID_ARG;
+  // Prefix pieces carry most of the bytes, and each is read once for up to 16
+  // query rows; long partitions keep their count (and the partials) low.
+  // Measured on B200 (shared-prefix workloads): 2048 beats 1024 and 512.
+  s->P = partition_size > 0 ? partition_size : std::max(2048, auto_partition(B, Hkv, max_seq_len));
+  const int64_t mp = std::max<int64_t>(1, ceil_div(max_seq_len, s->P));
+  if (mp > 32767) return PKV_ERR_OUT_OF_RANGE;
+  s->max_pp = (int)mp;
+  s->max_op = (int)mp;
+  s->SL = 2 * (int)mp;
+  const size_t G = (size_t)(Hq / Hkv);
+  const size_t units = (size_t)B * Hkv;
+  auto align256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  s->off_ml = align256(units * sizeof(uint32_t));
+  s->off_acc = s->off_ml + align256(units * s->SL * G * sizeof(float2));
+  s->bytes = B == 0 ? 0 : s->off_acc + units * s->SL * G * (size_t)D * sizeof(float);
+  return PKV_OK;
+}
+
+template <int D>
+int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap& mk,
+                  const CUtensorMap& mv, cudaStream_t stream) {
+  using C = pkv::MmaConsumer<D, 2>;
+  auto kernel = pkv::paged_decode_shared_kernel<C, D>;
+  const size_t smem = pkv::DecodeSmem<C>::kBytes;
+  static std::atomic<uint64_t> smem_set{0};
+  int rc = ensure_smem(kernel, smem, smem_set);
+  if (rc != PKV_OK) return rc;
+  kernel<<<(unsigned)items, pkv::kWarps * 32, smem, stream>>>(sp, mk, mv);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PKV_OK : cuda_fail(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -349,6 +394,100 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
   }
   if (D == 64) return dispatch_simt<float, 64>(p, bal, mk, mv, stream);
   return dispatch_simt<float, 128>(p, bal, mk, mv, stream);
+}
+
+size_t paged_attention_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D,
+                                                           int max_seq_len, int block_size,
+                                                           int partition_size) {
+  SharedShape s;
+  if (shared_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &s) != PKV_OK) return 0;
+  return s.bytes;
+}
+
+int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         int max_blocks, const int32_t* seq_lens, int max_seq_len,
+                                         const int32_t* group_offsets, const int32_t* prefix_lens,
+                                         int n_groups, int max_group_size, int B, int Hq, int Hkv,
+                                         int D, int block_size, int64_t num_blocks, float scale,
+                                         pkv_dtype dtype, int partition_size, void* workspace,
+                                         size_t workspace_bytes, pkv_stream_t stream) {
+  if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
+  SharedShape shape;
+  int rc = shared_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape);
+  if (rc != PKV_OK) return rc;
+  if (max_blocks <= 0 || num_blocks <= 0 || !std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+  if (n_groups <= 0 || max_group_size <= 0) return PKV_ERR_INVALID_ARG;
+  if (B == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !group_offsets ||
+      !prefix_lens)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+      (reinterpret_cast<uintptr_t>(group_offsets) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_lens) & 3u))
+    return PKV_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256) return PKV_ERR_UNSUPPORTED;
+  if (block_size % pkv::kStageTokens != 0 || block_size > 256) return PKV_ERR_UNSUPPORTED;
+  if (G > 16) return PKV_ERR_UNSUPPORTED;
+  if (num_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
+  if ((int64_t)max_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
+  if ((int64_t)max_seq_len > (int64_t)max_blocks * block_size) return PKV_ERR_OUT_OF_RANGE;
+  if (max_group_size > B) max_group_size = B;
+  if (shape.bytes > 0) {
+    if (!workspace || workspace_bytes < shape.bytes) return PKV_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
+  }
+  const int mc = std::max(1, 16 / G);
+  const int64_t chunks = ceil_div(max_group_size, mc);
+  const int64_t prefix_items = (int64_t)n_groups * chunks * shape.max_pp * Hkv;
+  const int64_t items = prefix_items + (int64_t)B * shape.max_op * Hkv;
+  if (items > 0x7fffffffLL) return PKV_ERR_OUT_OF_RANGE;
+
+  pkv::SharedParams sp;
+  pkv::DecodeParams& p = sp.d;
+  p.out = out;
+  p.q = q;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.ws_acc = nullptr;
+  p.ws_ml = nullptr;
+  p.ws_count = nullptr;
+  p.B = B;
+  p.max_blocks = max_blocks;
+  p.max_seq_len = max_seq_len;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.bs = block_size;
+  p.part_tokens = shape.P;
+  p.max_parts = shape.max_op;
+  p.num_blocks = (int)num_blocks;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  sp.group_offsets = group_offsets;
+  sp.prefix_lens = prefix_lens;
+  sp.ws_count = reinterpret_cast<uint32_t*>(ws);
+  sp.ws_ml = reinterpret_cast<float2*>(ws + shape.off_ml);
+  sp.ws_acc = reinterpret_cast<float*>(ws + shape.off_acc);
+  sp.n_groups = n_groups;
+  sp.chunks = (int)chunks;
+  sp.mc = mc;
+  sp.max_pp = shape.max_pp;
+  sp.max_op = shape.max_op;
+  sp.P = shape.P;
+  sp.n_prefix_items = (int)prefix_items;
+
+  CUtensorMap mk, mv;
+  const int64_t rows = num_blocks * block_size;
+  if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
+  if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
+  if (D == 64) return launch_shared<64>(sp, items, mk, mv, stream);
+  if (D == 128) return launch_shared<128>(sp, items, mk, mv, stream);
+  return launch_shared<256>(sp, items, mk, mv, stream);
 }
 
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int64_t P,

@@ -326,6 +326,37 @@ struct MmaConsumer {
     }
   }
 
+  // Rows n = i * G + g of the N dimension gather query head kvh * G + g of
+  // sequence b0 + i, for i < members (the members of a shared-prefix group).
+  __device__ __forceinline__ void init_gather(const DecodeParams& p, int b0, int members,
+                                              int kvh, int lane) {
+    const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+    scale_log2 = p.scale_log2;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int n = nt * 8 + lane / 4;
+      const int i = n / p.G, g = n % p.G;
+      const bool valid = i < members;
+      const uint32_t* row = reinterpret_cast<const uint32_t*>(
+          q + ((size_t)(b0 + (valid ? i : 0)) * p.Hq + (size_t)kvh * p.G + g) * D);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int d0 = ks * 16 + 2 * (lane % 4);
+        qf[nt][ks][0] = valid ? row[d0 / 2] : 0u;
+        qf[nt][ks][1] = valid ? row[(d0 + 8) / 2] : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        m[nt][j] = -INFINITY;
+        l[nt][j] = 0.f;
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) o[nt][mt][j] = 0.f;
+    }
+  }
+
   static __device__ __forceinline__ void load_stage(uint8_t* st, const CUtensorMap* tk,
                                                     const CUtensorMap* tv, uint64_t* bar,
                                                     int kvh, int row, uint64_t pol) {

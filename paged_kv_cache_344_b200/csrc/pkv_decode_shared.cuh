@@ -1,0 +1,329 @@
+// Shared-prefix decode (sm_100a): blocks shared by several sequences are read
+// once for all of them.
+//
+// Physical blocks may be shared between sequences -- decode branches of one
+// request, parallel samples, a common prompt -- through identical block-table
+// entries ("PagedAttention: paging the KV cache like an OS pages memory", How
+// it works).  The plain decode reads a shared block once per sequence.  Here
+// the caller lists groups of consecutive sequences whose first prefix_len
+// tokens sit in the same physical blocks, and the work is cut into
+//  * prefix pieces: (group, member chunk, prefix partition, KV head).  One CTA
+//    reads the partition's K/V once and scores it against the queries of up
+//    to 16 / G members at once: their G heads each stack into the N dimension
+//    of the tensor-core MMA (16 rows);
+//  * own pieces: (sequence, own partition, KV head) over the tokens after the
+//    prefix, exactly as in the plain decode.
+// Every piece leaves a partial (max, sum, weighted V) per (sequence, head); the
+// piece whose atomic ticket comes last for a (sequence, KV head) merges them
+// with a log-sum-exp rescale.  The result is the same softmax attention.
+//
+// Robustness: the prefix used for a group is shortened to the shortest
+// member's length and rounded down to 16 tokens; a prefix piece checks that
+// every member's table entries for its blocks equal the first member's.  A
+// mismatch, or group offsets that do not cover the batch, flags
+// PKV_DEVERR_PREFIX (results are then unreliable; memory stays in bounds).
+#pragma once
+
+#include "pkv_decode.cuh"
+
+namespace pkv {
+
+struct SharedParams {
+  DecodeParams d;                // out, q, tables, lengths, shapes, scale
+  const int32_t* group_offsets;  // [n_groups + 1]: group g = sequences off[g] .. off[g+1]-1
+  const int32_t* prefix_lens;    // [n_groups]
+  float* ws_acc;                 // [B*Hkv][slots][G][D]
+  float2* ws_ml;                 // [B*Hkv][slots][G]
+  uint32_t* ws_count;            // [B*Hkv]
+  int n_groups;
+  int chunks;     // member chunks per group (ceil(max group size / mc))
+  int mc;         // members per prefix piece: max(1, 16 / G)
+  int max_pp;     // prefix partitions per group (upper bound)
+  int max_op;     // own partitions per sequence (upper bound)
+  int P;          // partition length (tokens, multiple of 16)
+  int n_prefix_items;
+};
+
+__device__ __forceinline__ int shared_len(const DecodeParams& d, int b) {
+  const int cap = min(d.max_blocks * d.bs, d.max_seq_len);
+  const int L = d.seq_lens[b];
+  return L < 0 ? 0 : (L > cap ? cap : L);
+}
+
+// Prefix actually shared by group g: at most every member's length, whole stages.
+__device__ __forceinline__ int group_prefix(const SharedParams& s, int g, int lo, int hi) {
+  int plen = s.prefix_lens[g];
+  int minL = 0x7fffffff;
+  for (int b = lo; b < hi; ++b) minL = min(minL, shared_len(s.d, b));
+  if (hi <= lo) minL = 0;
+  plen = max(0, min(plen, minL));
+  return plen & ~(kStageTokens - 1);
+}
+
+// Group offset g clamped into [0, B]: offsets are caller data, and no value of
+// theirs may lead outside the batch.
+__device__ __forceinline__ int group_off(const SharedParams& s, int g) {
+  const int x = s.group_offsets[g];
+  return x < 0 ? 0 : (x > s.d.B ? s.d.B : x);
+}
+
+// Group of sequence b (binary search over the offsets); -1 if none covers b.
+__device__ __forceinline__ int group_of_seq(const SharedParams& s, int b) {
+  if (s.n_groups <= 0 || b < group_off(s, 0) || b >= group_off(s, s.n_groups)) return -1;
+  int lo = 0, hi = s.n_groups;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (group_off(s, mid) <= b) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+// What one CTA of the shared-prefix grid does.
+struct SharedItem {
+  bool valid;
+  bool prefix;
+  int kvh;
+  int b0;          // first sequence of the rows (prefix: first member of the chunk)
+  int members;     // rows are members x G (own pieces: 1)
+  int table_b;     // sequence whose table row gives the block ids
+  int t_begin, t_end;
+  int slot;        // partial slot of this piece for each of its sequences
+  int plen;        // shared prefix of the group (tokens)
+  int npp;         // prefix partitions of the group
+};
+
+__device__ __forceinline__ SharedItem decode_shared_item(const SharedParams& s, int x) {
+  SharedItem it;
+  it.valid = false;
+  it.prefix = x < s.n_prefix_items;
+  const int Hkv = s.d.Hkv;
+  it.kvh = x % Hkv;
+  int rest = x / Hkv;
+  if (it.prefix) {
+    const int pp = rest % s.max_pp;
+    rest /= s.max_pp;
+    const int c = rest % s.chunks;
+    const int g = rest / s.chunks;
+    const int lo = group_off(s, g), hi = max(lo, group_off(s, g + 1));
+    it.b0 = lo + c * s.mc;
+    it.members = min(s.mc, hi - it.b0);
+    if (it.members <= 0) return it;
+    it.plen = group_prefix(s, g, lo, hi);
+    it.npp = ceil_div_i(it.plen, s.P);
+    if (pp >= it.npp) return it;
+    it.table_b = lo;
+    it.t_begin = pp * s.P;
+    it.t_end = min(it.plen, it.t_begin + s.P);
+    it.slot = pp;
+  } else {
+    rest = (x - s.n_prefix_items) / Hkv;
+    const int op = rest % s.max_op;
+    const int b = rest / s.max_op;
+    const int g = group_of_seq(s, b);
+    if (g < 0) {
+      if (op == 0 && it.kvh == 0) flag_error(PKV_DEVERR_PREFIX);
+      it.plen = 0;
+      it.npp = 0;
+    } else {
+      const int lo = group_off(s, g);
+      it.plen = group_prefix(s, g, lo, max(lo, group_off(s, g + 1)));
+      it.npp = ceil_div_i(it.plen, s.P);
+    }
+    const int L = shared_len(s.d, b);
+    it.b0 = b;
+    it.members = 1;
+    it.table_b = b;
+    it.t_begin = it.plen + op * s.P;
+    it.t_end = min(L, it.t_begin + s.P);
+    // An empty sequence still needs its zero rows: own partition 0 writes them.
+    if (it.t_begin >= it.t_end && !(L == 0 && op == 0)) return it;
+    it.slot = s.max_pp + op;
+  }
+  it.valid = true;
+  return it;
+}
+
+// Pieces that contribute to (b, kvh): the group's prefix partitions + own ones.
+__device__ __forceinline__ int pieces_of(const SharedParams& s, int b, int plen, int npp) {
+  const int L = shared_len(s.d, b);
+  return npp + ceil_div_i(max(L - plen, 0), s.P);
+}
+
+template <class C, int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    paged_decode_shared_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
+                               const __grid_constant__ CUtensorMap tmV) {
+  using T = __nv_bfloat16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr int kRing = DecodeSmem<C>::kRingBytes;
+  static_assert(kRing >= (2 * C::GP + C::GP * D) * 4, "state does not fit in the ring");
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kRing);
+  __shared__ float s_M[16], s_den[16];
+  __shared__ int s_last;
+
+  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  const DecodeParams& p = s.d;
+  const SharedItem it = decode_shared_item(s, blockIdx.x);
+  if (!it.valid) return;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = p.G, kvh = it.kvh, Hkv = p.Hkv;
+  T* out = reinterpret_cast<T*>(p.out);
+  if (it.t_begin >= it.t_end) {  // an empty sequence: zero rows
+    T* o = out + ((size_t)it.b0 * p.Hq + (size_t)kvh * G) * D;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) o[i] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const int32_t* bt_row = p.block_tables + (size_t)it.table_b * p.max_blocks;
+  if (it.prefix) {  // every member must hold the same physical blocks for the prefix
+    const int j0 = it.t_begin / p.bs, j1 = (it.t_end - 1) / p.bs;
+    const int nj = j1 - j0 + 1;
+    for (int x = threadIdx.x; x < nj * it.members; x += blockDim.x) {
+      const int j = j0 + x % nj, b = it.b0 + x / nj;
+      if (p.block_tables[(size_t)b * p.max_blocks + j] != bt_row[j]) flag_error(PKV_DEVERR_PREFIX);
+    }
+  }
+
+  const int t_begin = it.t_begin, t_end = it.t_end;
+  const int n_st = (t_end - t_begin + kStageTokens - 1) / kStageTokens;
+  const int n_w = n_st > warp ? (n_st - warp + kWarps - 1) / kWarps : 0;
+  uint8_t* ring = smem + warp * kRing;
+  uint64_t* wbar = bars + warp * C::kStages;
+  if (lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+#pragma unroll
+    for (int st = 0; st < C::kStages; ++st) mbar_init(&wbar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t pol = l2_policy_evict_first();
+  auto stage_id = [&](int k) -> int {
+    return bt_row[(t_begin + (warp + kWarps * k) * kStageTokens) / p.bs];
+  };
+  int win_base = 0;
+  int win0 = lane < n_w ? stage_id(lane) : -1;
+  int win1 = 32 + lane < n_w ? stage_id(32 + lane) : -1;
+  auto issue = [&](int k) {
+    if (k - win_base >= 32) {
+      win0 = win1;
+      win_base += 32;
+      win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane) : -1;
+    }
+    const int id = __shfl_sync(kFull, win0, k - win_base);  // k - win_base < 32 here
+    if (lane == 0) {
+      const int st = k % C::kStages;
+      const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
+      int row;
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PKV_DEVERR_BLOCK_ID);
+        row = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
+      } else {
+        row = id * p.bs + t0 % p.bs;
+      }
+      mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
+      C::load_stage(ring + st * C::kStageBytes, &tmK, &tmV, &wbar[st], kvh, row, pol);
+    }
+  };
+  const int n_pro = n_w < C::kStages ? n_w : C::kStages;
+  for (int k = 0; k < n_pro; ++k) issue(k);
+
+  C c;
+  if (it.prefix) c.init_gather(p, it.b0, it.members, kvh, lane);
+  else c.init(p, it.b0, kvh, lane);
+  for (int k = 0; k < n_w; ++k) {
+    const int st = k % C::kStages;
+    const bool ok = mbar_wait_bounded(&wbar[st], (uint32_t)((k / C::kStages) & 1));
+    if (__any_sync(kFull, !ok)) {
+      if (lane == 0) flag_error(PKV_DEVERR_TIMEOUT);
+      for (int j = k; j < n_w && j < k + C::kStages; ++j)
+        mbar_wait_bounded(&wbar[j % C::kStages], (uint32_t)((j / C::kStages) & 1));
+      break;
+    }
+    const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
+    c.consume(ring + st * C::kStageBytes, min(kStageTokens, t_end - t0), lane);
+    __syncwarp();
+    if (k + C::kStages < n_w) issue(k + C::kStages);
+  }
+
+  // Merge the warps; each row n = member * G + head goes to its sequence.
+  c.store_state(reinterpret_cast<float*>(ring), lane);
+  __syncthreads();
+  constexpr int GP = C::GP;
+  const int rows = it.members * G;
+  const int SL = s.max_pp + s.max_op;
+  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
+    const int n = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, reinterpret_cast<const float*>(smem + w * kRing)[n]);
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float* stt = reinterpret_cast<const float*>(smem + w * kRing);
+      const float f = exp2f(stt[n] - M);
+      num = fmaf(f, stt[2 * GP + n * D + d], num);
+      den = fmaf(f, stt[GP + n], den);
+    }
+    const int b = it.b0 + n / G, gg = n % G;
+    if (pieces_of(s, b, it.plen, it.npp) == 1) {
+      out[((size_t)b * p.Hq + (size_t)kvh * G + gg) * D + d] = __float2bfloat16_rn(num / den);
+    } else {
+      const size_t u = (((size_t)b * Hkv + kvh) * SL + it.slot) * G + gg;
+      s.ws_acc[u * D + d] = num;
+      if (d == 0) s.ws_ml[u] = make_float2(M, den);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+
+  // Tickets: the last piece of each (sequence, KV head) merges its partials.
+  for (int i = 0; i < it.members; ++i) {
+    const int b = it.b0 + i;
+    const int tot = pieces_of(s, b, it.plen, it.npp);
+    if (tot <= 1) continue;
+    const size_t unit = (size_t)b * Hkv + kvh;
+    if (threadIdx.x == 0) s_last = atomicAdd(&s.ws_count[unit], 1u) == (uint32_t)(tot - 1);
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const size_t base = unit * SL * G;
+      auto slot_of = [&](int q) { return q < it.npp ? q : s.max_pp + (q - it.npp); };
+      for (int g = warp; g < G; g += kWarps) {
+        float M = -INFINITY;
+        for (int q = lane; q < tot; q += 32) M = fmaxf(M, __ldcg(&s.ws_ml[base + (size_t)slot_of(q) * G + g]).x);
+#pragma unroll
+        for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+        float den = 0.f;
+        for (int q = lane; q < tot; q += 32) {
+          const float2 ml = __ldcg(&s.ws_ml[base + (size_t)slot_of(q) * G + g]);
+          den += exp2f(ml.x - M) * ml.y;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
+        if (lane == 0) {
+          s_M[g] = M;
+          s_den[g] = den;
+        }
+      }
+      __syncthreads();
+      T* o = out + ((size_t)b * p.Hq + (size_t)kvh * G) * D;
+      for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+        const int g = idx / D, d = idx % D;
+        float num = 0.f;
+        for (int q = 0; q < tot; ++q) {
+          const size_t u = base + (size_t)slot_of(q) * G + g;
+          num = fmaf(exp2f(__ldcg(&s.ws_ml[u]).x - s_M[g]), __ldcg(&s.ws_acc[u * D + d]), num);
+        }
+        o[idx] = __float2bfloat16_rn(num / s_den[g]);
+      }
+      if (threadIdx.x == 0) s.ws_count[unit] = 0u;
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace pkv

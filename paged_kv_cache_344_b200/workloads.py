@@ -47,6 +47,10 @@ class Workload:
     seed: int
     scale: float = field(default=0.0)
     valid_pre: np.ndarray = field(default=None, repr=False)  # bool [NB, bs]: slot holds a token
+    # Groups of consecutive sequences whose first prefix_lens[g] tokens sit in the same
+    # physical blocks after the step (whole shared blocks; one-member groups share nothing).
+    group_offsets: np.ndarray = field(default=None, repr=False)  # int32 [n_groups + 1]
+    prefix_lens: np.ndarray = field(default=None, repr=False)  # int32 [n_groups]
 
     @property
     def G(self) -> int:
@@ -155,10 +159,23 @@ def _build(name, dtype, B, Hq, Hkv, D, bs, seq_lens_pre, seed, rng, pool_factor=
         bt[b, :len(ids)] = ids
         slot[b] = int(ids[lb]) * bs + off
 
+    # Group table: runs of equal group ids; the prefix is the whole blocks still shared
+    # by every member after the step (a partially filled shared block is copied on write).
+    starts = [0] + [b for b in range(1, B) if groups[b] != groups[b - 1]]
+    offsets = np.array(starts + [B], dtype=np.int32)
+    plens = []
+    for i, b in enumerate(starts):
+        g = int(groups[b])
+        members = range(b, int(offsets[i + 1]))
+        n_full = int(shared_tokens[g]) // bs if len(members) > 1 else 0
+        while n_full > 0 and len({int(bt[m, n_full - 1]) for m in members}) != 1:
+            n_full -= 1
+        plens.append(n_full * bs)
     wl = Workload(name=name, dtype=dtype, B=B, Hq=Hq, Hkv=Hkv, D=D, bs=bs, num_blocks=num_blocks,
                   seq_lens_pre=seq_lens_pre, block_tables_pre=bt_pre, block_tables=bt,
                   slot_mapping=slot, cow_pairs=np.asarray(cow, dtype=np.int64).reshape(-1, 2),
-                  seed=seed, valid_pre=valid)
+                  seed=seed, valid_pre=valid, group_offsets=offsets,
+                  prefix_lens=np.asarray(plens, dtype=np.int32))
     wl.scale = float(np.float32(1.0 / math.sqrt(D)))
     return wl
 
@@ -223,6 +240,20 @@ def custom(name, dtype, B, Hq, Hkv, D, bs, seq_lens_pre, seed, pool_factor=1.25,
     rng = np.random.default_rng(seed)
     return _build(name, dtype, B, Hq, Hkv, D, bs, np.asarray(seq_lens_pre), seed, rng,
                   pool_factor=pool_factor, min_pool=min_pool)
+
+
+def grouped(name, dtype, Hq, Hkv, D, bs, group_sizes, shared_tokens, tails, seed,
+            pool_factor=1.25):
+    """Groups of consecutive sequences that share a prefix of ``shared_tokens[g]`` tokens
+    (same physical blocks), each member followed by ``tails[b]`` tokens of its own."""
+    rng = np.random.default_rng(seed)
+    groups = np.repeat(np.arange(len(group_sizes)), group_sizes)
+    shared = np.asarray(shared_tokens, dtype=np.int64)
+    # Members write their own tokens after the prefix, so it must end on a block boundary.
+    assert np.all(shared % bs == 0), "shared prefixes must be whole blocks"
+    L = shared[groups] + np.asarray(tails, dtype=np.int64)
+    return _build(name, dtype, len(groups), Hq, Hkv, D, bs, L, seed, rng,
+                  pool_factor=pool_factor, groups=groups, shared_tokens=shared)
 
 
 def _to_bf16_bits(x: np.ndarray) -> np.ndarray:

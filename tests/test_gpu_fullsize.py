@@ -19,7 +19,9 @@ from gpu_util import assert_attention_close, gpu_step, meta_to_device, raw, to_h
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["mha", "gqa16", "gqa32", "long", "share_fork", "share_tails"]
+FULL = [("mha", False), ("gqa16", False), ("gqa32", False), ("long", False),
+        ("share_fork", False), ("share_tails", False), ("share_fork", True),
+        ("share_tails", True)]
 
 
 def _sample_units(wl, rng, n):
@@ -29,8 +31,9 @@ def _sample_units(wl, rng, n):
     return [(int(b), int(rng.integers(0, wl.Hkv))) for b in bs]
 
 
-@pytest.mark.parametrize("name", FULL)
-def test_fullsize_step(name):
+@pytest.mark.parametrize("name,shared", FULL,
+                         ids=[f"{n}{'-shared_prefix' if sh else ''}" for n, sh in FULL])
+def test_fullsize_step(name, shared):
     torch.cuda.empty_cache()
     pkv.device_errors(clear=True)
     wl = workloads.make(name)
@@ -52,7 +55,7 @@ def test_fullsize_step(name):
     before_all = {k: dev[k].clone() for k in ("k_cache", "v_cache")}
     host_new = {k: to_host_bits(dev[k]) for k in ("q", "k_new", "v_new")}
 
-    out = gpu_step(wl, dev)
+    out = gpu_step(wl, dev, shared=shared)
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0
 
