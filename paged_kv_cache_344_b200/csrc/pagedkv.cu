@@ -266,12 +266,15 @@ int shared_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
   return PKV_OK;
 }
 
-template <int D>
+// Prefix pieces stack up to 16 query rows (two 8-row MMA tiles); own pieces
+// need only G rows, so they run the one-tile consumer when G <= 8.
+template <int D, int NT_OWN>
 int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap& mk,
                   const CUtensorMap& mv, cudaStream_t stream) {
-  using C = pkv::MmaConsumer<D, 2>;
-  auto kernel = pkv::paged_decode_shared_kernel<C, D>;
-  const size_t smem = pkv::DecodeSmem<C>::kBytes;
+  using C2 = pkv::MmaConsumer<D, 2>;
+  using C1 = pkv::MmaConsumer<D, NT_OWN>;
+  auto kernel = pkv::paged_decode_shared_kernel<C2, C1, D>;
+  const size_t smem = pkv::DecodeSmem<C2>::kBytes;
   static std::atomic<uint64_t> smem_set{0};
   int rc = ensure_smem(kernel, smem, smem_set);
   if (rc != PKV_OK) return rc;
@@ -444,7 +447,7 @@ int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k
   const int mc = std::max(1, 16 / G);
   const int64_t chunks = ceil_div(max_group_size, mc);
   const int64_t prefix_items = (int64_t)n_groups * chunks * shape.max_pp * Hkv;
-  const int64_t items = prefix_items + (int64_t)B * shape.max_op * Hkv;
+  const int64_t items = prefix_items + (int64_t)n_groups * max_group_size * shape.max_op * Hkv;
   if (items > 0x7fffffffLL) return PKV_ERR_OUT_OF_RANGE;
 
   pkv::SharedParams sp;
@@ -478,6 +481,7 @@ int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k
   sp.mc = mc;
   sp.max_pp = shape.max_pp;
   sp.max_op = shape.max_op;
+  sp.max_group = max_group_size;
   sp.P = shape.P;
   sp.n_prefix_items = (int)prefix_items;
 
@@ -485,9 +489,14 @@ int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k
   const int64_t rows = num_blocks * block_size;
   if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
   if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
-  if (D == 64) return launch_shared<64>(sp, items, mk, mv, stream);
-  if (D == 128) return launch_shared<128>(sp, items, mk, mv, stream);
-  return launch_shared<256>(sp, items, mk, mv, stream);
+  if (G <= 8) {
+    if (D == 64) return launch_shared<64, 1>(sp, items, mk, mv, stream);
+    if (D == 128) return launch_shared<128, 1>(sp, items, mk, mv, stream);
+    return launch_shared<256, 1>(sp, items, mk, mv, stream);
+  }
+  if (D == 64) return launch_shared<64, 2>(sp, items, mk, mv, stream);
+  if (D == 128) return launch_shared<128, 2>(sp, items, mk, mv, stream);
+  return launch_shared<256, 2>(sp, items, mk, mv, stream);
 }
 
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int64_t P,

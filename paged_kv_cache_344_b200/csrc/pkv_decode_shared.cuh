@@ -40,6 +40,7 @@ struct SharedParams {
   int mc;         // members per prefix piece: max(1, 16 / G)
   int max_pp;     // prefix partitions per group (upper bound)
   int max_op;     // own partitions per sequence (upper bound)
+  int max_group;  // largest group size (upper bound)
   int P;          // partition length (tokens, multiple of 16)
   int n_prefix_items;
 };
@@ -67,15 +68,8 @@ __device__ __forceinline__ int group_off(const SharedParams& s, int g) {
   return x < 0 ? 0 : (x > s.d.B ? s.d.B : x);
 }
 
-// Group of sequence b (binary search over the offsets); -1 if none covers b.
-__device__ __forceinline__ int group_of_seq(const SharedParams& s, int b) {
-  if (s.n_groups <= 0 || b < group_off(s, 0) || b >= group_off(s, s.n_groups)) return -1;
-  int lo = 0, hi = s.n_groups;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (group_off(s, mid) <= b) lo = mid; else hi = mid;
-  }
-  return lo;
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
@@ -118,19 +112,18 @@ __device__ __forceinline__ SharedItem decode_shared_item(const SharedParams& s, 
     it.t_end = min(it.plen, it.t_begin + s.P);
     it.slot = pp;
   } else {
+    // Own pieces are enumerated per group, (g, member j, own partition, KV head),
+    // so a piece finds its sequence from two offsets instead of a search.
     rest = (x - s.n_prefix_items) / Hkv;
     const int op = rest % s.max_op;
-    const int b = rest / s.max_op;
-    const int g = group_of_seq(s, b);
-    if (g < 0) {
-      if (op == 0 && it.kvh == 0) flag_error(PKV_DEVERR_PREFIX);
-      it.plen = 0;
-      it.npp = 0;
-    } else {
-      const int lo = group_off(s, g);
-      it.plen = group_prefix(s, g, lo, max(lo, group_off(s, g + 1)));
-      it.npp = ceil_div_i(it.plen, s.P);
-    }
+    rest /= s.max_op;
+    const int j = rest % s.max_group;
+    const int g = rest / s.max_group;
+    const int lo = group_off(s, g), hi = max(lo, group_off(s, g + 1));
+    const int b = lo + j;
+    if (b >= hi) return it;
+    it.plen = group_prefix(s, g, lo, hi);
+    it.npp = ceil_div_i(it.plen, s.P);
     const int L = shared_len(s.d, b);
     it.b0 = b;
     it.members = 1;
@@ -151,24 +144,18 @@ __device__ __forceinline__ int pieces_of(const SharedParams& s, int b, int plen,
   return npp + ceil_div_i(max(L - plen, 0), s.P);
 }
 
+// One piece, run with consumer C (16 query rows for prefix pieces, the
+// smallest that holds G rows for own pieces).
 template <class C, int D>
-__global__ void __launch_bounds__(kWarps * 32)
-    paged_decode_shared_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
-                               const __grid_constant__ CUtensorMap tmV) {
+__device__ __forceinline__ void shared_piece(const SharedParams& s, const SharedItem& it,
+                                             uint8_t* smem, const CUtensorMap& tmK,
+                                             const CUtensorMap& tmV, float* s_M, float* s_den,
+                                             int& s_last) {
   using T = __nv_bfloat16;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   constexpr int kRing = DecodeSmem<C>::kRingBytes;
   static_assert(kRing >= (2 * C::GP + C::GP * D) * 4, "state does not fit in the ring");
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kRing);
-  __shared__ float s_M[16], s_den[16];
-  __shared__ int s_last;
-
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
   const DecodeParams& p = s.d;
-  const SharedItem it = decode_shared_item(s, blockIdx.x);
-  if (!it.valid) return;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G, kvh = it.kvh, Hkv = p.Hkv;
   T* out = reinterpret_cast<T*>(p.out);
@@ -178,6 +165,18 @@ __global__ void __launch_bounds__(kWarps * 32)
     return;
   }
   const int32_t* bt_row = p.block_tables + (size_t)it.table_b * p.max_blocks;
+  // Start the q rows and this piece's table entries on their way to L2 now.
+  {
+    const char* qrow = reinterpret_cast<const char*>(p.q) +
+                       ((size_t)it.b0 * p.Hq + (size_t)kvh * G) * D * sizeof(T);
+    const int lines = G * D * (int)sizeof(T) / 128;  // 128-byte lines of one member's rows
+    if ((int)threadIdx.x < it.members * lines) {
+      const int i = threadIdx.x / lines, line = threadIdx.x % lines;
+      prefetch_l2_line(qrow + (size_t)i * p.Hq * D * sizeof(T) + (size_t)line * 128);
+    }
+    const int tb0 = it.t_begin / p.bs, tb1 = (it.t_end - 1) / p.bs;
+    for (int j = tb0 + 32 * (int)threadIdx.x; j <= tb1; j += 32 * blockDim.x) prefetch_l2_line(bt_row + j);
+  }
   if (it.prefix) {  // every member must hold the same physical blocks for the prefix
     const int j0 = it.t_begin / p.bs, j1 = (it.t_end - 1) / p.bs;
     const int nj = j1 - j0 + 1;
@@ -324,6 +323,28 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     __syncthreads();
   }
+}
+
+template <class C2, class C1, int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    paged_decode_shared_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
+                               const __grid_constant__ CUtensorMap tmV) {
+  static_assert(DecodeSmem<C2>::kBytes == DecodeSmem<C1>::kBytes, "consumers share the ring");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ float s_M[16], s_den[16];
+  __shared__ int s_last;
+  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {  // the groups must tile the batch in order
+    bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
+    for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
+    if (!ok) flag_error(PKV_DEVERR_PREFIX);
+  }
+  const SharedItem it = decode_shared_item(s, blockIdx.x);
+  if (!it.valid) return;
+  if (it.prefix) shared_piece<C2, D>(s, it, smem, tmK, tmV, s_M, s_den, s_last);
+  else shared_piece<C1, D>(s, it, smem, tmK, tmV, s_M, s_den, s_last);
 }
 
 }  // namespace pkv
