@@ -234,7 +234,8 @@ def run_ours(args, rank, world, local_rank):
     pkv.set_decode_path({"auto": pkv.PKV_PATH_AUTO, "cuda_cores": pkv.PKV_PATH_CUDA_CORES,
                          "tensor_cores": pkv.PKV_PATH_TENSOR_CORES}[args.path])
     pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED if args.split == "balanced" else pkv.PKV_SPLIT_FIXED)
-    wl = workloads.make(args.config)
+    wl = workloads.make(args.config, block_size=args.block_size or None,
+                        contiguous=args.contiguous)
     dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
     meta = {
         "block_tables": torch.from_numpy(wl.block_tables).to(dev_name),
@@ -414,7 +415,8 @@ def run_ours(args, rank, world, local_rank):
                 "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                 "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
                 "decode_us": round(dec_avg_ms * 1e3, 2),
-                "algorithmic_bytes_per_launch": decode_bytes}
+                "algorithmic_bytes_per_launch": decode_bytes,
+                "achieved_token_exact": round(workloads.decode_token_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9, 1)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -443,6 +445,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "decode_entry": "paged_attention_decode_shared_prefix" if use_shared
                    else "paged_attention_decode",
+                   "block_size": wl.bs, "placement": "contiguous" if args.contiguous else "shuffled",
                    "decode_path": args.path, "decode_split": args.split,
                    "partition_tokens": part},
         "roofline": roofline,
@@ -507,6 +510,10 @@ def main():
     ap.add_argument("--decode", choices=["auto", "plain", "shared_prefix"], default="auto",
                     help="decode entry point (auto: shared-prefix decode for the shared-prefix "
                          "workloads, the plain decode otherwise)")
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="override the workload's block size (block-size sweep)")
+    ap.add_argument("--contiguous", action="store_true",
+                    help="lay each sequence's blocks out consecutively (contiguous-cache control)")
     ap.add_argument("--split", choices=["fixed", "balanced"], default="fixed",
                     help="decode work split (library default: fixed-length partitions)")
     ap.add_argument("--partition", type=int, default=0,

@@ -83,8 +83,9 @@ def _ceil_div(a: int, b: int) -> int:
 
 
 def _build(name, dtype, B, Hq, Hkv, D, bs, seq_lens_pre, seed, rng, pool_factor=1.25,
-           min_pool=0, groups=None, shared_tokens=None):
-    """Assign physical blocks for every sequence from a shuffled pool.
+           min_pool=0, groups=None, shared_tokens=None, contiguous=False):
+    """Assign physical blocks for every sequence from a shuffled pool (``contiguous``: in
+    pool order, so each sequence's blocks are consecutive, as in a contiguous cache).
 
     ``groups`` (optional) lists, per sequence, a group id; sequences of one group share the
     physical blocks of their first ``shared_tokens[group]`` tokens (refcount = group size).
@@ -105,6 +106,8 @@ def _build(name, dtype, B, Hq, Hkv, D, bs, seq_lens_pre, seed, rng, pool_factor=
         unique_need += int(need_post[b] - n_shared[groups[b]]) + 1  # +1: a possible CoW copy
     num_blocks = max(int(math.ceil(pool_factor * unique_need)), min_pool, 1)
     perm = rng.permutation(num_blocks).astype(np.int64)
+    if contiguous:
+        perm = np.arange(num_blocks, dtype=np.int64)
     cursor = 0
 
     def take(n):
@@ -186,14 +189,18 @@ CONFIG_INDEX = {"tiny": 0, "tiny_post": 0, "mha": 1, "gqa16": 2, "gqa32": 2, "lo
                 "share_fork": 4, "share_tails": 4}
 
 
-def make(name: str, seed: int | None = None, scale_down: int = 1) -> Workload:
+def make(name: str, seed: int | None = None, scale_down: int = 1, block_size: int | None = None,
+         contiguous: bool = False) -> Workload:
     """Build a named workload.
 
     Full-size names: ``tiny`` (lengths are pre-step), ``tiny_post`` (lengths include the
     new token), ``mha``, ``gqa16``, ``gqa32``, ``long``, ``share_fork``, ``share_tails``.
     ``scale_down > 1`` divides the batch and the lengths for fast parity tests while keeping
-    the head shapes, block size and length distribution.
+    the head shapes, block size and length distribution.  ``block_size`` overrides the
+    workload's block size; ``contiguous`` lays every sequence's blocks out consecutively
+    (a contiguous-cache control for the cost of the scattered placement).
     """
+    kw = {"contiguous": contiguous}
     if seed is None:
         seed = 1000 + CONFIG_INDEX[name]
     rng = np.random.default_rng(seed)
@@ -206,18 +213,18 @@ def make(name: str, seed: int | None = None, scale_down: int = 1) -> Workload:
     if name == "mha":
         B = max(64 // s, 2)
         L = rng.integers(128 // s, 2048 // s + 1, size=B)
-        return _build(name, "bf16", B, 40, 40, 128, 16, L, seed, rng)
+        return _build(name, "bf16", B, 40, 40, 128, block_size or 16, L, seed, rng, **kw)
     if name in ("gqa16", "gqa32"):
-        bs = 16 if name == "gqa16" else 32
+        bs = block_size or (16 if name == "gqa16" else 32)
         B = max(256 // s, 2)
         z = rng.standard_normal(B)
         L = np.clip(np.round(np.exp(math.log(1024) + 0.8 * z)), 16, 4096).astype(np.int64) // s
         L = np.maximum(L, 1)
-        return _build(name, "bf16", B, 32, 8, 128, bs, L, seed, rng)
+        return _build(name, "bf16", B, 32, 8, 128, bs, L, seed, rng, **kw)
     if name == "long":
         B = max(8 // s, 1)
         L = rng.integers(32768 // s, 131072 // s + 1, size=B)
-        return _build(name, "bf16", B, 64, 8, 128, 16, L, seed, rng)
+        return _build(name, "bf16", B, 64, 8, 128, block_size or 16, L, seed, rng, **kw)
     if name in ("share_fork", "share_tails"):
         n_groups, branches = max(32 // s, 1), 4
         B = n_groups * branches
@@ -326,6 +333,20 @@ def decode_algorithmic_bytes(wl: Workload) -> int:
     qo = 2 * wl.B * wl.Hq * wl.D * wl.elt
     tables = sum(_ceil_div(int(n), wl.bs) for n in wl.seq_lens_post) * 4
     return int(kv + qo + tables + 4 * wl.B)
+
+
+def decode_token_bytes(wl: Workload) -> int:
+    """Like ``decode_algorithmic_bytes`` but counting only the cached tokens themselves (no
+    unused slots of the last blocks; shared tokens once per group)."""
+    row = wl.Hkv * wl.D * wl.elt * 2
+    tokens = int(wl.seq_lens_post.sum())
+    if wl.group_offsets is not None:
+        for g in range(len(wl.prefix_lens)):
+            n = int(wl.group_offsets[g + 1] - wl.group_offsets[g])
+            tokens -= (n - 1) * int(wl.prefix_lens[g])
+    qo = 2 * wl.B * wl.Hq * wl.D * wl.elt
+    tables = sum(_ceil_div(int(n), wl.bs) for n in wl.seq_lens_post) * 4
+    return int(tokens * row + qo + tables + 4 * wl.B)
 
 
 def write_bytes(wl: Workload) -> int:
