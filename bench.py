@@ -259,13 +259,35 @@ def run_ours(args, rank, world, local_rank):
     ws = torch.zeros(max(ws_bytes, 1), dtype=torch.uint8, device=dev_name)
     out = torch.empty_like(dev["q"])
     has_cow = len(wl.cow_pairs) > 0
-    launches_per_step = 2 + int(has_cow)
+    launches_per_step = 1 if args.step == "fused" else 2 + int(has_cow)
     stream = torch.cuda.current_stream()
 
     # The CoW step restores its own precondition: copying block src -> dst again is
     # idempotent, and rewriting the same token to the same slot is too.
+    fused = args.step == "fused"
+    if fused:
+        meta["cow_src"] = torch.from_numpy(wl.cow_src).to(dev_name)
+
     def step(d_in, ev_pair=None, outbuf=None):
         o = out if outbuf is None else outbuf
+        if fused:
+            if ev_pair is not None:
+                ev_pair[0].record(stream)
+            cow = d_in["cow_src"] if has_cow else None
+            if use_shared:
+                pkv.paged_decode_step_shared_prefix(
+                    o, d_in["q"], d_in["k_new"], d_in["v_new"], d_in["k_cache"],
+                    d_in["v_cache"], d_in["block_tables"], d_in["seq_lens"], wl.max_seq_len,
+                    wl.scale, d_in["group_offsets"], d_in["prefix_lens"], max_group,
+                    cow_src=cow, workspace=ws, partition_size=args.partition)
+            else:
+                pkv.paged_decode_step(o, d_in["q"], d_in["k_new"], d_in["v_new"], d_in["k_cache"],
+                                      d_in["v_cache"], d_in["block_tables"], d_in["seq_lens"],
+                                      wl.max_seq_len, wl.scale, cow_src=cow, workspace=ws,
+                                      partition_size=args.partition)
+            if ev_pair is not None:
+                ev_pair[1].record(stream)
+            return
         if has_cow:
             pkv.copy_blocks(d_in["k_cache"], d_in["v_cache"], d_in["cow_pairs"])
         pkv.paged_kv_write(d_in["k_new"], d_in["v_new"], d_in["k_cache"], d_in["v_cache"],
@@ -346,7 +368,7 @@ def run_ours(args, rank, world, local_rank):
     # step i's output run on a copy stream and overlap the computation of step i (two sets
     # of step buffers; the KV cache itself stays resident).
     in_keys = [k for k in ("q", "k_new", "v_new", "block_tables", "seq_lens", "slot_mapping",
-                           "cow_pairs", "group_offsets", "prefix_lens")
+                           "cow_pairs", "group_offsets", "prefix_lens", "cow_src")
                if k in d_in and (k != "cow_pairs" or has_cow)]
     host_in = {k: d_in[k].cpu().pin_memory() for k in in_keys}
     bufs = [dict(d_in), dict(d_in)]
@@ -404,10 +426,12 @@ def run_ours(args, rank, world, local_rank):
 
     peak, peak_src = load_peaks()
     dec_avg_ms = statistics.fmean(dec_ms)
-    achieved = decode_bytes / (dec_avg_ms * 1e-3) / 1e9
+    kernel_bytes = step_bytes if fused else decode_bytes  # the fused kernel also writes/copies
+    achieved = kernel_bytes / (dec_avg_ms * 1e-3) / 1e9
     G = wl.G
     tc = wl.dtype == "bf16" and (args.path != "cuda_cores" or G > 8)
     kernel = ("paged_decode_shared_kernel" if use_shared else
+              "paged_decode_kernel" if fused else
               "paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
         + ("<MmaConsumer>" if tc else "<SimtConsumer>")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
@@ -415,7 +439,7 @@ def run_ours(args, rank, world, local_rank):
                 "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                 "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
                 "decode_us": round(dec_avg_ms * 1e3, 2),
-                "algorithmic_bytes_per_launch": decode_bytes,
+                "algorithmic_bytes_per_launch": kernel_bytes,
                 "achieved_token_exact": round(workloads.decode_token_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9, 1)}
 
     cpu = None
@@ -438,7 +462,11 @@ def run_ours(args, rank, world, local_rank):
         "pct_of_8TBps_spec": round(100 * value / world / SPEC_HBM_GBS, 2),
         "pct_of_measured_peak": round(100 * value / world / peak, 2),
         "config": {"workload": args.config, "description": DESCR.get(args.config, args.config),
-                   "step": ("copy_blocks + " if has_cow else "") + "paged_kv_write + paged_attention_decode",
+                   "step": (("paged_decode_step_shared_prefix" if use_shared else "paged_decode_step")
+                            + " (copy-on-write + cache write + decode in one launch)" if fused else
+                            ("copy_blocks + " if has_cow else "") + "paged_kv_write + "
+                            + ("paged_attention_decode_shared_prefix" if use_shared
+                               else "paged_attention_decode")),
                    "bytes_per_step": step_bytes,
                    "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
                           else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
@@ -514,6 +542,9 @@ def main():
                     help="override the workload's block size (block-size sweep)")
     ap.add_argument("--contiguous", action="store_true",
                     help="lay each sequence's blocks out consecutively (contiguous-cache control)")
+    ap.add_argument("--step", choices=["separate", "fused"], default="fused",
+                    help="run the step as one fused launch (paged_decode_step[_shared_prefix]) "
+                         "or as copy_blocks + paged_kv_write + decode")
     ap.add_argument("--split", choices=["fixed", "balanced"], default="fixed",
                     help="decode work split (library default: fixed-length partitions)")
     ap.add_argument("--partition", type=int, default=0,

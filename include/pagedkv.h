@@ -162,6 +162,36 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
                            pkv_stream_t stream);
 
 /*
+ * paged_decode_step: one whole decode step in one launch.  For every sequence b
+ * with L = seq_lens[b] > 0, in this order:
+ *   1. if cow_src != NULL and cow_src[b] >= 0: copy physical block cow_src[b] into
+ *      the block that holds token L - 1 (block_tables[b][(L-1) / block_size]),
+ *      as copy_blocks does;
+ *   2. store k_new[b], v_new[b] as token L - 1, as paged_kv_write does with
+ *      slot = block_tables[b][(L-1) / block_size] * block_size + (L-1) % block_size;
+ *   3. decode as paged_attention_decode over tokens 0 .. L-1.
+ * This is the per-step loop of the pages: cache the new token, copying a shared
+ * block before modifying it ([Explained] "Step 2" and "Step 4"; [Wiki] "How it
+ * works").  The copy and the write are done, per KV head, by the decode CTA of
+ * the sequence's last partition, which is the only CTA that reads that block.
+ * So one launch replaces three.
+ *   seq_lens  lengths after the step (they include the new token)
+ *   k_new, v_new  device [B][Hkv][D]
+ *   cow_src   device [B] int32 or NULL; -1 = no copy
+ * Contract: the copy targets only blocks that receive this step's new tokens
+ * (copy-on-write of a shared block about to be written).  The other arguments,
+ * the workspace rules and the supported shapes are those of
+ * paged_attention_decode, with fixed-length partitions whatever
+ * pkv_set_decode_split says.
+ */
+int paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
+                      void *k_cache, void *v_cache, const int32_t *block_tables, int max_blocks,
+                      const int32_t *seq_lens, const int32_t *cow_src, int max_seq_len, int B,
+                      int Hq, int Hkv, int D, int block_size, int64_t num_blocks, float scale,
+                      pkv_dtype dtype, int partition_size, void *workspace, size_t workspace_bytes,
+                      pkv_stream_t stream);
+
+/*
  * paged_attention_decode_shared_prefix: paged_attention_decode for batches in
  * which consecutive sequences share the physical blocks of a prefix: decode
  * branches of one request, parallel samples, a common prompt.  Physical blocks
@@ -178,7 +208,7 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
  *   prefix_lens    device [n_groups] int32: leading tokens whose blocks are
  *                  the same physical blocks in every member (equal table
  *                  entries).  The decode uses min(prefix_len, shortest member's
- *                  length), rounded down to a multiple of 16.  0 means nothing shared.
+ *                  length - 1), rounded down to a multiple of 16.  0 means nothing shared.
  *   max_group_size host upper bound of the group sizes.
  * The other arguments are as for paged_attention_decode.  bf16 only, G <= 16.
  * The workspace (paged_attention_decode_shared_prefix_workspace_size) follows the
@@ -195,6 +225,25 @@ int paged_attention_decode_shared_prefix(void *out, const void *q, const void *k
                                          int D, int block_size, int64_t num_blocks, float scale,
                                          pkv_dtype dtype, int partition_size, void *workspace,
                                          size_t workspace_bytes, pkv_stream_t stream);
+
+/*
+ * paged_decode_step_shared_prefix: paged_decode_step for grouped batches.  It
+ * does the copy-on-write copy and the new token's write, then
+ * paged_attention_decode_shared_prefix, all in one launch.  The new token
+ * (position seq_lens[b] - 1) must lie after the group's shared prefix; the decode
+ * caps the prefix one token short of the shortest member, so that holds for any
+ * prefix_lens value.  Arguments are those of the two calls.
+ */
+int paged_decode_step_shared_prefix(void *out, const void *q, const void *k_new,
+                                    const void *v_new, void *k_cache, void *v_cache,
+                                    const int32_t *block_tables, int max_blocks,
+                                    const int32_t *seq_lens, const int32_t *cow_src,
+                                    int max_seq_len, const int32_t *group_offsets,
+                                    const int32_t *prefix_lens, int n_groups, int max_group_size,
+                                    int B, int Hq, int Hkv, int D, int block_size,
+                                    int64_t num_blocks, float scale, pkv_dtype dtype,
+                                    int partition_size, void *workspace, size_t workspace_bytes,
+                                    pkv_stream_t stream);
 
 /* Workspace bytes of paged_attention_decode_shared_prefix (pure host function;
  * 0 for invalid arguments). */

@@ -78,6 +78,13 @@ def lib() -> ctypes.CDLL:
     L.paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
                                          i32, i64, f32, i32, i32, vp, sz, vp]
     L.paged_attention_decode.restype = i32
+    L.paged_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
+                                    i32, i32, i64, f32, i32, i32, vp, sz, vp]
+    L.paged_decode_step.restype = i32
+    L.paged_decode_step_shared_prefix.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32,
+                                                  vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                                  i64, f32, i32, i32, vp, sz, vp]
+    L.paged_decode_step_shared_prefix.restype = i32
     L.paged_attention_decode_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
                                                  i32, i32, i32, i64, f32, i32, i32, vp]
     L.paged_attention_decode_noalloc.restype = i32
@@ -171,6 +178,38 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, max
         block_tables.shape[1], _ptr(seq_lens), int(max_seq_len), B, Hq, Hkv, D, bs, NB,
         float(scale), _dtype_code(q), int(partition_size), _ptr(workspace), ws_bytes,
         _stream(q, stream)))
+
+
+def paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens,
+                      max_seq_len, scale, cow_src=None, workspace=None, partition_size=0,
+                      stream=None) -> None:
+    """One decode step in one launch: optional copy-on-write of each sequence's last block
+    (``cow_src[b]``), cache write of its new token (position ``seq_lens[b] - 1``), decode."""
+    B, Hq, D = q.shape
+    NB, bs, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("paged_decode_step", lib().paged_decode_step(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), _ptr(cow_src),
+        int(max_seq_len), B, Hq, Hkv, D, bs, NB, float(scale), _dtype_code(q),
+        int(partition_size), _ptr(workspace), ws_bytes, _stream(q, stream)))
+
+
+def paged_decode_step_shared_prefix(out, q, k_new, v_new, k_cache, v_cache, block_tables,
+                                    seq_lens, max_seq_len, scale, group_offsets, prefix_lens,
+                                    max_group_size, cow_src=None, workspace=None,
+                                    partition_size=0, stream=None) -> None:
+    """paged_decode_step for grouped batches: copy-on-write, cache write and the
+    shared-prefix decode in one launch."""
+    B, Hq, D = q.shape
+    NB, bs, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("paged_decode_step_shared_prefix", lib().paged_decode_step_shared_prefix(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), block_tables.shape[1], _ptr(seq_lens), _ptr(cow_src),
+        int(max_seq_len), _ptr(group_offsets), _ptr(prefix_lens), prefix_lens.shape[0],
+        int(max_group_size), B, Hq, Hkv, D, bs, NB, float(scale), _dtype_code(q),
+        int(partition_size), _ptr(workspace), ws_bytes, _stream(q, stream)))
 
 
 def paged_attention_decode_noalloc(out, q, k_cache, v_cache, block_tables, seq_lens, max_seq_len,

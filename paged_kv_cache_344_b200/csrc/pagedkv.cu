@@ -116,7 +116,7 @@ struct DecodeShape {
 };
 
 int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
-                 int partition_size, DecodeShape* s) {
+                 int partition_size, DecodeShape* s, bool force_fixed = false) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || max_seq_len < 0)
     return PKV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
@@ -146,7 +146,8 @@ int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
     b_acc = b_ml + align256(slots * G * sizeof(float2));
     b_bytes = b_acc + slots * G * (size_t)D * sizeof(float);
   }
-  s->balanced = bal_ok && g_decode_split.load(std::memory_order_relaxed) == PKV_SPLIT_BALANCED;
+  s->balanced = bal_ok && !force_fixed &&
+                g_decode_split.load(std::memory_order_relaxed) == PKV_SPLIT_BALANCED;
   s->P = s->balanced ? 0 : P;
   s->max_parts = s->balanced ? 0 : (int)mp;
   s->off_ml = s->balanced ? b_ml : f_ml;
@@ -327,14 +328,27 @@ size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int 
   return s.ws_bytes;
 }
 
-int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                           const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
-                           int max_seq_len, int B, int Hq, int Hkv, int D, int block_size,
-                           int64_t num_blocks, float scale, pkv_dtype dtype, int partition_size,
-                           void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused step's extra inputs (all null for a plain decode).
+struct StepArgs {
+  const void* k_new = nullptr;
+  const void* v_new = nullptr;
+  const int32_t* cow_src = nullptr;
+};
+
+int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                int max_seq_len, int B, int Hq, int Hkv, int D, int block_size,
+                int64_t num_blocks, float scale, pkv_dtype dtype, int partition_size,
+                void* workspace, size_t workspace_bytes, pkv_stream_t stream,
+                const StepArgs& step) {
+  const bool fused = step.k_new != nullptr;
   if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
   DecodeShape shape;
-  int rc = decode_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape);
+  int rc = decode_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape, fused);
   if (rc != PKV_OK) return rc;
   if (max_blocks <= 0 || num_blocks <= 0 || !std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
   if (B == 0) return PKV_OK;
@@ -357,7 +371,10 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PKV_ERR_WORKSPACE;
   }
 
-  pkv::DecodeParams p;
+  if (fused && (!step.v_new || !aligned16(step.k_new) || !aligned16(step.v_new) ||
+                (reinterpret_cast<uintptr_t>(step.cow_src) & 3u)))
+    return PKV_ERR_INVALID_ARG;
+  pkv::DecodeParams p{};
   p.out = out;
   p.q = q;
   p.block_tables = block_tables;
@@ -377,6 +394,13 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
   p.max_parts = shape.max_parts;
   p.num_blocks = (int)num_blocks;
   p.scale_log2 = scale * 1.4426950408889634f;
+  if (fused) {
+    p.k_new = step.k_new;
+    p.v_new = step.v_new;
+    p.k_cache_w = const_cast<void*>(k_cache);
+    p.v_cache_w = const_cast<void*>(v_cache);
+    p.cow_src = step.cow_src;
+  }
 
   const bool tc = use_tensor_cores(dtype, G);
   CUtensorMap mk, mv;
@@ -399,6 +423,36 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
   return dispatch_simt<float, 128>(p, bal, mk, mv, stream);
 }
 
+}  // namespace
+
+extern "C" {
+
+int paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                           const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                           int max_seq_len, int B, int Hq, int Hkv, int D, int block_size,
+                           int64_t num_blocks, float scale, pkv_dtype dtype, int partition_size,
+                           void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks, seq_lens, max_seq_len, B,
+                     Hq, Hkv, D, block_size, num_blocks, scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, StepArgs{});
+}
+
+int paged_decode_step(void* out, const void* q, const void* k_new, const void* v_new,
+                      void* k_cache, void* v_cache, const int32_t* block_tables, int max_blocks,
+                      const int32_t* seq_lens, const int32_t* cow_src, int max_seq_len, int B,
+                      int Hq, int Hkv, int D, int block_size, int64_t num_blocks, float scale,
+                      pkv_dtype dtype, int partition_size, void* workspace, size_t workspace_bytes,
+                      pkv_stream_t stream) {
+  if (!k_new || !v_new) return PKV_ERR_INVALID_ARG;
+  StepArgs step;
+  step.k_new = k_new;
+  step.v_new = v_new;
+  step.cow_src = cow_src;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks, seq_lens, max_seq_len, B,
+                     Hq, Hkv, D, block_size, num_blocks, scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, step);
+}
+
 size_t paged_attention_decode_shared_prefix_workspace_size(int B, int Hq, int Hkv, int D,
                                                            int max_seq_len, int block_size,
                                                            int partition_size) {
@@ -407,14 +461,17 @@ size_t paged_attention_decode_shared_prefix_workspace_size(int B, int Hq, int Hk
   return s.bytes;
 }
 
-int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_cache,
-                                         const void* v_cache, const int32_t* block_tables,
-                                         int max_blocks, const int32_t* seq_lens, int max_seq_len,
-                                         const int32_t* group_offsets, const int32_t* prefix_lens,
-                                         int n_groups, int max_group_size, int B, int Hq, int Hkv,
-                                         int D, int block_size, int64_t num_blocks, float scale,
-                                         pkv_dtype dtype, int partition_size, void* workspace,
-                                         size_t workspace_bytes, pkv_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int shared_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
+                const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                int max_seq_len, const int32_t* group_offsets, const int32_t* prefix_lens,
+                int n_groups, int max_group_size, int B, int Hq, int Hkv, int D, int block_size,
+                int64_t num_blocks, float scale, pkv_dtype dtype, int partition_size,
+                void* workspace, size_t workspace_bytes, pkv_stream_t stream,
+                const StepArgs& step) {
   if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
   SharedShape shape;
   int rc = shared_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape);
@@ -450,8 +507,16 @@ int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k
   const int64_t items = prefix_items + (int64_t)n_groups * max_group_size * shape.max_op * Hkv;
   if (items > 0x7fffffffLL) return PKV_ERR_OUT_OF_RANGE;
 
-  pkv::SharedParams sp;
+  if (step.k_new && (!step.v_new || !aligned16(step.k_new) || !aligned16(step.v_new) ||
+                     (reinterpret_cast<uintptr_t>(step.cow_src) & 3u)))
+    return PKV_ERR_INVALID_ARG;
+  pkv::SharedParams sp{};
   pkv::DecodeParams& p = sp.d;
+  p.k_new = step.k_new;
+  p.v_new = step.v_new;
+  p.k_cache_w = step.k_new ? const_cast<void*>(k_cache) : nullptr;
+  p.v_cache_w = step.k_new ? const_cast<void*>(v_cache) : nullptr;
+  p.cow_src = step.cow_src;
   p.out = out;
   p.q = q;
   p.block_tables = block_tables;
@@ -497,6 +562,44 @@ int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k
   if (D == 64) return launch_shared<64, 2>(sp, items, mk, mv, stream);
   if (D == 128) return launch_shared<128, 2>(sp, items, mk, mv, stream);
   return launch_shared<256, 2>(sp, items, mk, mv, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attention_decode_shared_prefix(void* out, const void* q, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         int max_blocks, const int32_t* seq_lens, int max_seq_len,
+                                         const int32_t* group_offsets, const int32_t* prefix_lens,
+                                         int n_groups, int max_group_size, int B, int Hq, int Hkv,
+                                         int D, int block_size, int64_t num_blocks, float scale,
+                                         pkv_dtype dtype, int partition_size, void* workspace,
+                                         size_t workspace_bytes, pkv_stream_t stream) {
+  return shared_impl(out, q, k_cache, v_cache, block_tables, max_blocks, seq_lens, max_seq_len,
+                     group_offsets, prefix_lens, n_groups, max_group_size, B, Hq, Hkv, D,
+                     block_size, num_blocks, scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, StepArgs{});
+}
+
+int paged_decode_step_shared_prefix(void* out, const void* q, const void* k_new, const void* v_new,
+                                    void* k_cache, void* v_cache, const int32_t* block_tables,
+                                    int max_blocks, const int32_t* seq_lens, const int32_t* cow_src,
+                                    int max_seq_len, const int32_t* group_offsets,
+                                    const int32_t* prefix_lens, int n_groups, int max_group_size,
+                                    int B, int Hq, int Hkv, int D, int block_size,
+                                    int64_t num_blocks, float scale, pkv_dtype dtype,
+                                    int partition_size, void* workspace, size_t workspace_bytes,
+                                    pkv_stream_t stream) {
+  if (!k_new || !v_new) return PKV_ERR_INVALID_ARG;
+  StepArgs step;
+  step.k_new = k_new;
+  step.v_new = v_new;
+  step.cow_src = cow_src;
+  return shared_impl(out, q, k_cache, v_cache, block_tables, max_blocks, seq_lens, max_seq_len,
+                     group_offsets, prefix_lens, n_groups, max_group_size, B, Hq, Hkv, D,
+                     block_size, num_blocks, scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, step);
 }
 
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int64_t P,

@@ -58,6 +58,14 @@ struct DecodeParams {
   int max_parts;
   int num_blocks;
   float scale_log2;  // scale * log2(e)
+  // Fused step (paged_decode_step): the CTA of a sequence's last partition first
+  // copies the copy-on-write source block and writes the new token (position
+  // L - 1), both for its own KV head.  Null k_new: plain decode.
+  const void* k_new;     // [B][Hkv][D]
+  const void* v_new;
+  void* k_cache_w;       // the caches, written by the fused step
+  void* v_cache_w;
+  const int32_t* cow_src;  // [B] or null: block copied into the new token's block first
 };
 
 template <typename T>
@@ -532,6 +540,51 @@ struct MmaConsumer {
 };
 
 // ---------------------------------------------------------------------------
+// Fused step: the cache update of token L - 1 of sequence b for KV head kvh,
+// after the copy-on-write copy of its block when cow_src[b] >= 0 ("PagedAttention:
+// paging the KV cache like an OS pages memory", How it works: a shared block that
+// must be modified is copied first).  Only the CTA of the sequence's last
+// partition reads that block, so no other CTA needs these writes; the proxy fence
+// makes them visible to this CTA's TMA loads.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__device__ __forceinline__ void fused_append(const DecodeParams& p, int b, int kvh, int L) {
+  const int t = L - 1;
+  const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks;
+  const int dst = bt_row[t / p.bs];
+  if (dst < 0 || dst >= p.num_blocks) {
+    if (threadIdx.x == 0) flag_error(PKV_DEVERR_BLOCK_ID);
+    return;
+  }
+  constexpr int kVec = D * (int)sizeof(T) / 16;  // 16-byte vectors per head row
+  const size_t row_vec = (size_t)p.Hkv * kVec;    // per token row (all heads)
+  uint4* kc = reinterpret_cast<uint4*>(p.k_cache_w);
+  uint4* vc = reinterpret_cast<uint4*>(p.v_cache_w);
+  const int src = p.cow_src != nullptr ? p.cow_src[b] : -1;
+  if (src >= p.num_blocks) {
+    if (threadIdx.x == 0) flag_error(PKV_DEVERR_COPY);
+  } else if (src >= 0 && src != dst) {
+    for (int i = threadIdx.x; i < p.bs * kVec; i += blockDim.x) {
+      const int r = i / kVec, c = i % kVec;
+      const size_t so = ((size_t)src * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
+      const size_t d_o = ((size_t)dst * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
+      kc[d_o] = kc[so];
+      vc[d_o] = vc[so];
+    }
+    __syncthreads();  // the copy lands before the new token's row overwrites it
+  }
+  const uint4* kn = reinterpret_cast<const uint4*>(p.k_new);
+  const uint4* vn = reinterpret_cast<const uint4*>(p.v_new);
+  for (int c = threadIdx.x; c < kVec; c += blockDim.x) {
+    const size_t d_o = ((size_t)dst * p.bs + t % p.bs) * row_vec + (size_t)kvh * kVec + c;
+    const size_t so = ((size_t)b * p.Hkv + kvh) * kVec + c;
+    kc[d_o] = kn[so];
+    vc[d_o] = vn[so];
+  }
+  fence_proxy_async_global();
+}
+
+// ---------------------------------------------------------------------------
 // The kernel skeleton shared by both consumers.
 // ---------------------------------------------------------------------------
 template <class C>
@@ -575,6 +628,10 @@ __global__ void __launch_bounds__(kWarps * 32)
     return;
   }
   if (part >= nparts) return;
+  if (p.k_new != nullptr && part == nparts - 1) {
+    fused_append<T, D>(p, b, kvh, L);
+    __syncthreads();
+  }
 
   const int t_begin = part * P;
   const int t_end = min(L, t_begin + P);

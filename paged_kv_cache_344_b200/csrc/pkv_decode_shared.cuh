@@ -17,8 +17,8 @@
 // piece whose atomic ticket comes last for a (sequence, KV head) merges them
 // with a log-sum-exp rescale.  The result is the same softmax attention.
 //
-// Robustness: the prefix used for a group is shortened to the shortest
-// member's length and rounded down to 16 tokens; a prefix piece checks that
+// Robustness: the prefix used for a group is shortened to one token less than
+// the shortest member and rounded down to 16 tokens; a prefix piece checks that
 // every member's table entries for its blocks equal the first member's.  A
 // mismatch, or group offsets that do not cover the batch, flags
 // PKV_DEVERR_PREFIX (results are then unreliable; memory stays in bounds).
@@ -51,11 +51,12 @@ __device__ __forceinline__ int shared_len(const DecodeParams& d, int b) {
   return L < 0 ? 0 : (L > cap ? cap : L);
 }
 
-// Prefix actually shared by group g: at most every member's length, whole stages.
+// Prefix actually shared by group g: short of every member's newest token (which
+// a fused step writes), whole stages.
 __device__ __forceinline__ int group_prefix(const SharedParams& s, int g, int lo, int hi) {
   int plen = s.prefix_lens[g];
   int minL = 0x7fffffff;
-  for (int b = lo; b < hi; ++b) minL = min(minL, shared_len(s.d, b));
+  for (int b = lo; b < hi; ++b) minL = min(minL, shared_len(s.d, b) - 1);
   if (hi <= lo) minL = 0;
   plen = max(0, min(plen, minL));
   return plen & ~(kStageTokens - 1);
@@ -163,6 +164,12 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
     T* o = out + ((size_t)it.b0 * p.Hq + (size_t)kvh * G) * D;
     for (int i = threadIdx.x; i < G * D; i += blockDim.x) o[i] = __float2bfloat16_rn(0.f);
     return;
+  }
+  if (!it.prefix && p.k_new != nullptr && it.t_end == shared_len(p, it.b0)) {
+    // Fused step: this own piece holds the sequence's new token (never inside the
+    // shared prefix), so it alone reads that token's block.
+    fused_append<T, D>(p, it.b0, kvh, it.t_end);
+    __syncthreads();
   }
   const int32_t* bt_row = p.block_tables + (size_t)it.table_b * p.max_blocks;
   // Start the q rows and this piece's table entries on their way to L2 now.

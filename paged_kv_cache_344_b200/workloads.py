@@ -69,6 +69,18 @@ class Workload:
         return int(self.seq_lens_post.max()) if self.B else 0
 
     @property
+    def cow_src(self) -> np.ndarray:
+        """Per sequence: the block copied into its new token's block this step, else -1."""
+        src = np.full(self.B, -1, dtype=np.int32)
+        by_dst = {int(d): int(s_) for s_, d in self.cow_pairs}
+        for b in range(self.B):
+            if self.slot_mapping[b] >= 0:
+                dst = int(self.slot_mapping[b]) // self.bs
+                if dst in by_dst:
+                    src[b] = by_dst[dst]
+        return src
+
+    @property
     def elt(self) -> int:
         return 2 if self.dtype == "bf16" else 4
 

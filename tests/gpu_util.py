@@ -57,9 +57,35 @@ def workspace_for(wl, partition_size=0, device="cuda"):
 
 
 def gpu_step(wl, dev, partition_size=0, workspace=None, max_seq_len=None, stream=None,
-             shared=False):
+             shared=False, fused=False):
     """copy_blocks -> paged_kv_write -> paged_attention_decode (or, with ``shared``, the
-    shared-prefix decode over the workload's groups) on the device; returns out."""
+    shared-prefix decode over the workload's groups; with ``fused``, paged_decode_step:
+    all three in one launch) on the device; returns out."""
+    if fused and shared:
+        out = torch.empty_like(dev["q"])
+        msl = max_seq_len or wl.max_seq_len
+        n = pkv.paged_attention_decode_shared_prefix_workspace_size(
+            wl.B, wl.Hq, wl.Hkv, wl.D, msl, wl.bs, partition_size)
+        ws = torch.zeros(max(n, 1), dtype=torch.uint8, device=dev["q"].device)
+        cow = torch.from_numpy(wl.cow_src).to(dev["q"].device) if len(wl.cow_pairs) else None
+        pkv.paged_decode_step_shared_prefix(
+            out, dev["q"], dev["k_new"], dev["v_new"], dev["k_cache"], dev["v_cache"],
+            dev["block_tables"], dev["seq_lens"], msl, wl.scale,
+            torch.from_numpy(wl.group_offsets).to(dev["q"].device),
+            torch.from_numpy(wl.prefix_lens).to(dev["q"].device),
+            int(np.diff(wl.group_offsets).max()), cow_src=cow, workspace=ws,
+            partition_size=partition_size, stream=stream)
+        return out
+    if fused:
+        out = torch.empty_like(dev["q"])
+        if workspace is None:
+            workspace = workspace_for(wl, partition_size)
+        cow = torch.from_numpy(wl.cow_src).to(dev["q"].device) if len(wl.cow_pairs) else None
+        pkv.paged_decode_step(out, dev["q"], dev["k_new"], dev["v_new"], dev["k_cache"],
+                              dev["v_cache"], dev["block_tables"], dev["seq_lens"],
+                              max_seq_len or wl.max_seq_len, wl.scale, cow_src=cow,
+                              workspace=workspace, partition_size=partition_size, stream=stream)
+        return out
     if len(wl.cow_pairs):
         pkv.copy_blocks(dev["k_cache"], dev["v_cache"], dev["cow_pairs"], stream=stream)
     pkv.paged_kv_write(dev["k_new"], dev["v_new"], dev["k_cache"], dev["v_cache"],

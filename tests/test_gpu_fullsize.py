@@ -19,9 +19,10 @@ from gpu_util import assert_attention_close, gpu_step, meta_to_device, raw, to_h
 
 pytestmark = pytest.mark.gpu
 
-FULL = [("mha", False), ("gqa16", False), ("gqa32", False), ("long", False),
-        ("share_fork", False), ("share_tails", False), ("share_fork", True),
-        ("share_tails", True)]
+FULL = [("mha", ""), ("gqa16", ""), ("gqa32", ""), ("long", ""), ("share_fork", ""),
+        ("share_tails", ""), ("share_fork", "shared_prefix"), ("share_tails", "shared_prefix"),
+        ("mha", "fused_step"), ("long", "fused_step"), ("share_fork", "fused_step"),
+        ("share_fork", "fused_shared_prefix"), ("share_tails", "fused_shared_prefix")]
 
 
 def _sample_units(wl, rng, n):
@@ -31,9 +32,8 @@ def _sample_units(wl, rng, n):
     return [(int(b), int(rng.integers(0, wl.Hkv))) for b in bs]
 
 
-@pytest.mark.parametrize("name,shared", FULL,
-                         ids=[f"{n}{'-shared_prefix' if sh else ''}" for n, sh in FULL])
-def test_fullsize_step(name, shared):
+@pytest.mark.parametrize("name,entry", FULL, ids=[f"{n}-{e}" if e else n for n, e in FULL])
+def test_fullsize_step(name, entry):
     torch.cuda.empty_cache()
     pkv.device_errors(clear=True)
     wl = workloads.make(name)
@@ -55,7 +55,7 @@ def test_fullsize_step(name, shared):
     before_all = {k: dev[k].clone() for k in ("k_cache", "v_cache")}
     host_new = {k: to_host_bits(dev[k]) for k in ("q", "k_new", "v_new")}
 
-    out = gpu_step(wl, dev, shared=shared)
+    out = gpu_step(wl, dev, shared=entry.endswith("shared_prefix"), fused=entry.startswith("fused"))
     torch.cuda.synchronize()
     assert pkv.device_errors() == 0
 
