@@ -12,6 +12,7 @@ wraps it with NumPy arrays:
 * ``kv_write(...)``: byte scatter of new tokens into their slots.
 * ``copy_blocks(...)``: whole-block copies for copy-on-write.
 * ``paged_decode(...)``: fp64 softmax attention over the block-table-resolved cache.
+* ``paged_prefill(...)``: the same for several causal queries per sequence.
 
 Element arrays are NumPy ``uint16`` (bf16 bit patterns) or ``float32``.
 """
@@ -75,6 +76,9 @@ class Oracle:
         lib.oracle_paged_decode.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, i64, vp, i64, i64,
                                             i64, i64, i64, i64, dp, vp, vp, i64]
         lib.oracle_paged_decode.restype = ctypes.c_int
+        lib.oracle_paged_prefill.argtypes = [vp, vp, vp, vp, ctypes.c_int, vp, i64, vp, vp, i64,
+                                             i64, i64, i64, i64, i64, dp]
+        lib.oracle_paged_prefill.restype = ctypes.c_int
         self.lib = lib
 
     def num_threads(self) -> int:
@@ -141,6 +145,29 @@ class Oracle:
         return out
 
 
+def _prefill(self, q, k_cache, v_cache, block_tables, seq_lens, cu_q, scale):
+    """fp64 multi-query attention: ``q [T,Hq,D]`` rows ``cu_q[b] .. cu_q[b+1]-1`` are the
+    last queries of sequence b, each attending causally.  Returns ``[T,Hq,D]`` float64."""
+    T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    assert D2 == D and v_cache.shape == k_cache.shape and q.dtype == k_cache.dtype
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    cq = np.ascontiguousarray(cu_q, dtype=np.int32)
+    B = sl.shape[0]
+    assert cq.shape == (B + 1,) and cq[-1] == T and bt.shape[0] == B
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = self.lib.oracle_paged_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       _dtype_code(q), _ptr(bt), bt.shape[1], _ptr(sl), _ptr(cq),
+                                       B, Hq, Hkv, D, bs, NB, float(scale))
+    if rc != 0:
+        raise ValueError(f"oracle_paged_prefill failed with status {rc}")
+    return out
+
+
+Oracle.paged_prefill = _prefill
+
+
 def default() -> Oracle:
     """The oracle built from ``pkv_oracle.c`` (compiled on first use)."""
     global _default
@@ -167,3 +194,7 @@ def copy_blocks(k_cache, v_cache, block_mapping) -> int:
 
 def paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, rows=None):
     return default().paged_decode(q, k_cache, v_cache, block_tables, seq_lens, scale, rows)
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, seq_lens, cu_q, scale):
+    return default().paged_prefill(q, k_cache, v_cache, block_tables, seq_lens, cu_q, scale)

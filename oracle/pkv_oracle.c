@@ -26,6 +26,9 @@
  *                            full).  slot < 0 means "no write".
  *   oracle_copy_blocks       block-granularity copy-on-write copies ([Wiki]
  *                            "How it works", second paragraph).
+ *   oracle_paged_prefill     multi-query (prefill / chunked append) attention:
+ *                            every query row is the decode definition over the
+ *                            tokens up to its own position (causal).
  *   oracle_paged_decode      single-query attention over the paged cache.
  *                            The attention itself is ordinary softmax
  *                            attention; only the storage layout differs
@@ -151,15 +154,13 @@ int64_t oracle_copy_blocks(void *k_cache, void *v_cache, const int64_t *mapping,
     return bad;
 }
 
-/* One output row: query head h of sequence b. */
-static int decode_row(double *out_row, const void *q, const void *k_cache, const void *v_cache,
-                      int dtype, const int32_t *block_tables, int64_t max_blocks,
-                      const int32_t *seq_lens, int64_t b, int64_t h, int64_t Hq, int64_t Hkv,
+/* One output row: the query at element offset q_off of q against the first L
+ * cached tokens of sequence b, KV head kvh. */
+static int attend_row(double *out_row, const void *q, int64_t q_off, const void *k_cache,
+                      const void *v_cache, int dtype, const int32_t *block_tables,
+                      int64_t max_blocks, int64_t b, int64_t L, int64_t kvh, int64_t Hkv,
                       int64_t D, int64_t bs, int64_t num_blocks, double scale)
 {
-    const int64_t G = Hq / Hkv;
-    const int64_t kvh = h / G;
-    const int64_t L = seq_lens[b];
     int64_t t, d;
 
     for (d = 0; d < D; ++d) out_row[d] = 0.0;
@@ -188,7 +189,7 @@ static int decode_row(double *out_row, const void *q, const void *k_cache, const
     double smax = -INFINITY;
     for (t = 0; t < L; ++t) {
         double acc = 0.0;
-        for (d = 0; d < D; ++d) acc += load_elem(q, (b * Hq + h) * D + d, dtype) * Kc[t * D + d];
+        for (d = 0; d < D; ++d) acc += load_elem(q, q_off + d, dtype) * Kc[t * D + d];
         s[t] = scale * acc;
         if (s[t] > smax) smax = s[t];
     }
@@ -205,6 +206,18 @@ static int decode_row(double *out_row, const void *q, const void *k_cache, const
 
     free(Kc); free(Vc); free(s);
     return 0;
+}
+
+/* Decode row: query head h of sequence b attends to all seq_lens[b] tokens. */
+static int decode_row(double *out_row, const void *q, const void *k_cache, const void *v_cache,
+                      int dtype, const int32_t *block_tables, int64_t max_blocks,
+                      const int32_t *seq_lens, int64_t b, int64_t h, int64_t Hq, int64_t Hkv,
+                      int64_t D, int64_t bs, int64_t num_blocks, double scale)
+{
+    const int64_t G = Hq / Hkv;
+    const int64_t kvh = h / G;
+    return attend_row(out_row, q, (b * Hq + h) * D, k_cache, v_cache, dtype, block_tables,
+                      max_blocks, b, seq_lens[b], kvh, Hkv, D, bs, num_blocks, scale);
 }
 
 /* Decode attention.  q: [B, Hq, D]; caches: [num_blocks, bs, Hkv, D];
@@ -228,6 +241,42 @@ int oracle_paged_decode(double *out, const void *q, const void *k_cache, const v
         const int64_t h = rows_b ? rows_h[r] : r % Hq;
         const int rc = decode_row(out + r * D, q, k_cache, v_cache, dtype, block_tables,
                                   max_blocks, seq_lens, b, h, Hq, Hkv, D, bs, num_blocks, scale);
+        if (rc != 0) {
+#pragma omp critical
+            status = rc;
+        }
+    }
+    return status;
+}
+
+/* Multi-query (prefill / chunked append) attention.  Sequence b holds
+ * L = seq_lens[b] tokens, the last Q = cu_q[b+1] - cu_q[b] of which are this
+ * call's queries, packed as rows cu_q[b] .. cu_q[b+1]-1 of q [T, Hq, D].  Query
+ * i of sequence b sits at position L - Q + i and attends causally, to tokens
+ * 0 .. L - Q + i: each row is the decode definition with that many tokens.
+ * out: [T, Hq, D] doubles.  Returns the first nonzero status of a row, -1 for
+ * bad dimensions or Q > L. */
+int oracle_paged_prefill(double *out, const void *q, const void *k_cache, const void *v_cache,
+                         int dtype, const int32_t *block_tables, int64_t max_blocks,
+                         const int32_t *seq_lens, const int32_t *cu_q, int64_t B, int64_t Hq,
+                         int64_t Hkv, int64_t D, int64_t bs, int64_t num_blocks, double scale)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || bs <= 0 || Hq % Hkv != 0) return -1;
+    const int64_t T = cu_q[B];
+    for (int64_t b = 0; b < B; ++b)
+        if (cu_q[b + 1] < cu_q[b] || cu_q[b + 1] - cu_q[b] > seq_lens[b]) return -1;
+    int status = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < T * Hq; ++r) {
+        const int64_t row = r / Hq, h = r % Hq;
+        int64_t b = 0;
+        while (cu_q[b + 1] <= row) ++b;
+        const int64_t Q = cu_q[b + 1] - cu_q[b];
+        const int64_t i = row - cu_q[b];
+        const int64_t visible = seq_lens[b] - Q + i + 1; /* causal: up to its own position */
+        const int64_t kv_head = h / (Hq / Hkv);
+        const int rc = attend_row(out + r * D, q, r * D, k_cache, v_cache, dtype, block_tables,
+                                  max_blocks, b, visible, kv_head, Hkv, D, bs, num_blocks, scale);
         if (rc != 0) {
 #pragma omp critical
             status = rc;

@@ -443,3 +443,71 @@ def test_row_selection_matches_full(o=None):
                           wl.scale, rows=rows)
     for i, (b, h) in enumerate(rows):
         np.testing.assert_array_equal(part[i], full[b, h])
+
+
+# --------------------------------------------------------------------------------------
+# Multi-query (prefill / chunked append) attention
+# --------------------------------------------------------------------------------------
+
+def _prefill_problem(seed, lens, qlens, Hq=4, Hkv=2, D=16, bs=16):
+    rng = np.random.default_rng(seed)
+    Ks = [rng.standard_normal((L, Hkv, D), dtype=np.float32) for L in lens]
+    Vs = [rng.standard_normal((L, Hkv, D), dtype=np.float32) for L in lens]
+    NB = sum(-(-L // bs) for L in lens) + 3
+    kc, vc, bt, sl = _pool_from(Ks, Vs, bs, NB, seed)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), Hq, D), dtype=np.float32)
+    return q, Ks, Vs, kc, vc, bt, sl, cu
+
+
+def test_prefill_single_query_equals_decode(o=None):
+    """With one query per sequence, the multi-query attention is the decode, bit for bit."""
+    o = _oracle(o)
+    q, Ks, Vs, kc, vc, bt, sl, cu = _prefill_problem(31, [5, 40, 17], [1, 1, 1])
+    pre = o.paged_prefill(q, kc, vc, bt, sl, cu, 0.3)
+    dec = o.paged_decode(q, kc, vc, bt, sl, 0.3)
+    np.testing.assert_array_equal(pre, dec)
+
+
+def test_prefill_equals_causal_sdpa_float64(o=None):
+    """Equals PyTorch's scaled_dot_product_attention in float64 with an explicit causal mask
+    on the contiguous tensors: query i of a chunk of Q sees tokens 0 .. L - Q + i."""
+    o = _oracle(o)
+    for seed, (Hq, Hkv) in enumerate([(4, 4), (8, 2), (6, 3)]):
+        lens, qlens = [33, 7, 64], [9, 7, 1]
+        q, Ks, Vs, kc, vc, bt, sl, cu = _prefill_problem(40 + seed, lens, qlens, Hq, Hkv, D=24)
+        out = o.paged_prefill(q, kc, vc, bt, sl, cu, 0.2)
+        G = Hq // Hkv
+        for b, (L, Q) in enumerate(zip(lens, qlens)):
+            K = torch.from_numpy(Ks[b]).double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+            V = torch.from_numpy(Vs[b]).double().repeat_interleave(G, dim=1).permute(1, 0, 2)[None]
+            qq = torch.from_numpy(q[cu[b]:cu[b + 1]]).double().permute(1, 0, 2)[None]  # [1,Hq,Q,D]
+            mask = torch.arange(L)[None, :] <= (L - Q + torch.arange(Q))[:, None]   # [Q, L]
+            ref = torch.nn.functional.scaled_dot_product_attention(qq, K, V, attn_mask=mask,
+                                                                   scale=0.2)
+            np.testing.assert_allclose(out[cu[b]:cu[b + 1]], ref[0].permute(1, 0, 2).numpy(),
+                                       rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_brute_force_tiny(o=None):
+    o = _oracle(o)
+    rng = np.random.default_rng(44)
+    for trial in range(6):
+        L = int(rng.integers(2, 6))
+        Q = int(rng.integers(1, L + 1))
+        D = int(rng.integers(1, 4))
+        q, Ks, Vs, kc, vc, bt, sl, cu = _prefill_problem(50 + trial, [L], [Q], Hq=1, Hkv=1, D=D,
+                                                         bs=2)
+        out = o.paged_prefill(q, kc, vc, bt, sl, cu, 0.7)
+        for i in range(Q):
+            vis = L - Q + i + 1
+            ref = _softmax_decimal(q[i, 0], Ks[0][:vis, 0], Vs[0][:vis, 0], 0.7)
+            np.testing.assert_allclose(out[i, 0], ref, rtol=1e-14, atol=1e-15)
+
+
+def test_prefill_rejects_chunks_longer_than_sequences(o=None):
+    o = _oracle(o)
+    q, Ks, Vs, kc, vc, bt, sl, cu = _prefill_problem(60, [5], [5])
+    o.paged_prefill(q, kc, vc, bt, sl, cu, 0.5)
+    with pytest.raises(ValueError):
+        o.paged_prefill(q, kc, vc, bt, np.array([4], np.int32), cu, 0.5)

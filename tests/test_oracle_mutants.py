@@ -23,7 +23,10 @@ MUTANTS = {
     "dropped_scale": ("s[t] = scale * acc;", "s[t] = acc;"),
     "dropped_normalisation": ("out_row[d] /= wsum;", "out_row[d] /= 1.0;"),
     "dropped_dot_term": ("for (d = 0; d < D; ++d) acc +=", "for (d = 1; d < D; ++d) acc +="),
-    "q_head_index": ("(b * Hq + h) * D + d", "(b * Hq + kvh) * D + d"),
+    "q_head_index": ("(b * Hq + h) * D, k_cache", "(b * Hq + kvh) * D, k_cache"),
+    "prefill_causal_bound": ("seq_lens[b] - Q + i + 1;", "seq_lens[b] - Q + i;"),
+    "prefill_kv_head": ("const int64_t kv_head = h / (Hq / Hkv);", "const int64_t kv_head = h % Hkv;"),
+    "prefill_q_row": ("attend_row(out + r * D, q, r * D,", "attend_row(out + r * D, q, row * D,"),
     "k_for_v_operand": ("out_row[d] += w * Vc[t * D + d];", "out_row[d] += w * Kc[t * D + d];"),
     "write_offset": ("const int64_t offset = s % bs;", "const int64_t offset = (s + 1) % bs;"),
     "write_block": ("const int64_t block = s / bs;", "const int64_t block = s / (bs + 1);"),
