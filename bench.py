@@ -491,6 +491,59 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def run_prefill(args, rank, world, local_rank):
+    """Multi-query (chunked append) attention on the tcgen05 kernel: TFLOP/s."""
+    import torch
+    import paged_kv_cache_344_b200 as pkv
+    torch.cuda.set_device(local_rank)
+    dev_name = f"cuda:{local_rank}"
+    wl, cu_q = workloads.prefill()
+    dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
+    T = int(cu_q[-1])
+    gen = torch.Generator(device=dev_name)
+    gen.manual_seed(4242 + rank)
+    q = torch.randn((T, wl.Hq, wl.D), generator=gen, device=dev_name).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    bt = torch.from_numpy(wl.block_tables).to(dev_name)
+    seq = torch.from_numpy(wl.seq_lens_pre).to(dev_name)
+    cu = torch.from_numpy(cu_q).to(dev_name)
+    max_q = int(np.diff(cu_q).max())
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pkv.paged_attention_prefill(out, q, dev["k_cache"], dev["v_cache"], bt, seq, cu, max_q,
+                                    int(wl.seq_lens_pre.max()), wl.scale)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev_name)
+    flops = workloads.prefill_flops(wl, cu_q)
+    tflops = world * flops / (ms * 1e-3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, src = float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (burst)"
+    except Exception:
+        peak, src = 1590.0, "fallback"
+    return {"metric": "paged multi-query (chunked append) attention: TFLOP/s",
+            "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prefill: B=16, chunk 512 appended to U{0..4096} cached tokens, "
+                                   "Hq=32, Hkv=8, D=128, bs=16", "flops_per_step": flops},
+            "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
+                         "traffic": None, "kernel": "paged_prefill_kernel", "peak_source": src},
+            "gpu_launches": args.steps, "clocks": clocks.summary()}
+
+
 def run_reference(args, rank, world):
     """The reference arm: the fp64 oracle on this host's cores, each step a bounded sample
     of the same workload."""
@@ -533,6 +586,8 @@ def main():
     ap.add_argument("--cpu-budget-rows", type=int, default=400_000_000,
                     help="query-row x token budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
+                    help="decode step (default) or multi-query chunked-append attention")
     ap.add_argument("--path", choices=["auto", "cuda_cores", "tensor_cores"], default="auto",
                     help="decode kernel family (library default: auto)")
     ap.add_argument("--decode", choices=["auto", "plain", "shared_prefix"], default="auto",
@@ -568,7 +623,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device(f"cuda:{local_rank}"))
     try:
-        line = run_ours(args, rank, world, local_rank)
+        line = (run_prefill(args, rank, world, local_rank) if args.mode == "prefill"
+                else run_ours(args, rank, world, local_rank))
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

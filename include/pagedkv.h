@@ -162,6 +162,29 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
                            pkv_stream_t stream);
 
 /*
+ * paged_attention_prefill: multi-query attention over the paged cache, for
+ * prefill or a chunked append.  Sequence b holds L = seq_lens[b] cached tokens,
+ * whose last Q = cu_q[b+1] - cu_q[b] are this call's queries (their K/V already
+ * written, e.g. by paged_kv_write).  Query i (row cu_q[b] + i of q) sits at
+ * position L - Q + i and attends causally to tokens 0 .. L - Q + i: each row is
+ * paged_attention_decode's softmax attention over its visible prefix ([Wiki]
+ * "How it works": standard causal attention, only the layout changes).
+ *   out, q        device [total_q][Hq][D]
+ *   cu_q          device [B + 1] int32, non-decreasing, cu_q[B] = total_q
+ *   max_q_len     host upper bound of Q; max_seq_len host upper bound of L
+ * It runs on the tcgen05 tensor cores.  Each CTA takes 128 query rows (128/G
+ * tokens x G heads of one KV head) and streams the sequence's K/V in 64-token
+ * tiles through TMEM accumulators.  bf16 only; G in {1, 2, 4, 8, 16}; D in
+ * {64, 128, 256}; block_size a multiple of 16 up to 256.  A sequence with Q > L
+ * flags PKV_DEVERR_SEQLEN and its rows are not written.
+ */
+int paged_attention_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, int max_blocks, const int32_t *seq_lens,
+                            const int32_t *cu_q, int total_q, int max_q_len, int max_seq_len,
+                            int B, int Hq, int Hkv, int D, int block_size, int64_t num_blocks,
+                            float scale, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
  * paged_decode_step: one whole decode step in one launch.  For every sequence b
  * with L = seq_lens[b] > 0, in this order:
  *   1. if cow_src != NULL and cow_src[b] >= 0: copy physical block cow_src[b] into

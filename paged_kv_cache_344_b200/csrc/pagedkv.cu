@@ -13,6 +13,7 @@
 
 #include "pkv_decode_balanced.cuh"
 #include "pkv_decode_shared.cuh"
+#include "pkv_prefill.cuh"
 #include "pkv_write_copy.cuh"
 
 namespace {
@@ -600,6 +601,85 @@ int paged_decode_step_shared_prefix(void* out, const void* q, const void* k_new,
                      group_offsets, prefix_lens, n_groups, max_group_size, B, Hq, Hkv, D,
                      block_size, num_blocks, scale, dtype, partition_size, workspace,
                      workspace_bytes, stream, step);
+}
+
+int paged_attention_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                            const int32_t* cu_q, int total_q, int max_q_len, int max_seq_len,
+                            int B, int Hq, int Hkv, int D, int block_size, int64_t num_blocks,
+                            float scale, pkv_dtype dtype, pkv_stream_t stream) {
+  if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
+  if (B < 0 || total_q < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 ||
+      max_blocks <= 0 || num_blocks <= 0 || max_seq_len < 0 || max_q_len < 0 ||
+      !std::isfinite(scale) || Hq % Hkv != 0)
+    return PKV_ERR_INVALID_ARG;
+  if (B == 0 || total_q == 0) return PKV_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !cu_q)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(cu_q) & 3u))
+    return PKV_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (D != 64 && D != 128 && D != 256) return PKV_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return PKV_ERR_UNSUPPORTED;
+  if (block_size % pkv::kStageTokens != 0 || block_size > 256) return PKV_ERR_UNSUPPORTED;
+  if (max_q_len < 1 || max_q_len > max_seq_len) return PKV_ERR_OUT_OF_RANGE;
+  if (num_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
+  if ((int64_t)max_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
+  if ((int64_t)max_seq_len > (int64_t)max_blocks * block_size) return PKV_ERR_OUT_OF_RANGE;
+  const int TQ = pkv::kPrefillRows / G;
+  const int64_t q_tiles = ceil_div(max_q_len, TQ);
+  if (B > 65535 || q_tiles > 65535) return PKV_ERR_OUT_OF_RANGE;
+
+  pkv::PrefillParams p{};
+  p.out = out;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.cu_q = cu_q;
+  p.max_blocks = max_blocks;
+  p.max_seq_len = max_seq_len;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = G;
+  p.TQ = TQ;
+  p.bs = block_size;
+  p.num_blocks = (int)num_blocks;
+  p.scale_log2 = scale * 1.4426950408889634f;
+
+  // Query rows [T][Hq][D] as a 3-D tensor {D, Hq, T}; one box = 128 rows of one
+  // KV head: {64, G, 128 / G}, 128-byte swizzled (the K-major MMA operand).
+  auto fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  CUtensorMap mq, mk, mv;
+  cuuint64_t qdims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)total_q};
+  cuuint64_t qstrides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+  cuuint32_t qbox[3] = {64u, (cuuint32_t)G, (cuuint32_t)TQ};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), qdims, qstrides,
+                  qbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = 100000 + static_cast<int>(r);
+    return PKV_ERR_CUDA;
+  }
+  int rc;
+  const int64_t rows = num_blocks * block_size;
+  if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
+  if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
+  dim3 grid((unsigned)Hkv, (unsigned)q_tiles, (unsigned)B);
+  auto launch = [&](auto kernel, size_t smem, std::atomic<uint64_t>& set) -> int {
+    int rc2 = ensure_smem(kernel, smem, set);
+    if (rc2 != PKV_OK) return rc2;
+    kernel<<<grid, pkv::kWarps * 32, smem, stream>>>(p, mq, mk, mv);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PKV_OK : cuda_fail(e);
+  };
+  static std::atomic<uint64_t> set64{0}, set128{0}, set256{0};
+  if (D == 64) return launch(pkv::paged_prefill_kernel<64>, pkv::PrefillSmem<64>::kBytes, set64);
+  if (D == 128) return launch(pkv::paged_prefill_kernel<128>, pkv::PrefillSmem<128>::kBytes, set128);
+  return launch(pkv::paged_prefill_kernel<256>, pkv::PrefillSmem<256>::kBytes, set256);
 }
 
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int64_t P,

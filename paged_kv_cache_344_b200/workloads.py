@@ -275,6 +275,28 @@ def grouped(name, dtype, Hq, Hkv, D, bs, group_sizes, shared_tokens, tails, seed
                   pool_factor=pool_factor, groups=groups, shared_tokens=shared)
 
 
+def prefill(seed: int = 1005, B: int = 16, chunk: int = 512, max_ctx: int = 4096, Hq: int = 32,
+            Hkv: int = 8, D: int = 128, bs: int = 16):
+    """A chunked-append batch: sequence b has ctx_b ~ U{0..max_ctx} cached tokens followed by
+    ``chunk`` new query tokens (already in the cache).  Returns (workload, cu_q) where the
+    workload's ``seq_lens_pre`` are the full lengths ctx_b + chunk."""
+    rng = np.random.default_rng(seed)
+    ctx = rng.integers(0, max_ctx + 1, size=B)
+    wl = custom("prefill", "bf16", B, Hq, Hkv, D, bs, ctx + chunk, seed)
+    cu_q = (np.arange(B + 1) * chunk).astype(np.int32)
+    return wl, cu_q
+
+
+def prefill_flops(wl: Workload, cu_q: np.ndarray) -> int:
+    """Multiply-add flops of causal multi-query attention: 4 D per (query row, visible token)."""
+    total = 0
+    for b in range(wl.B):
+        L, Q = int(wl.seq_lens_pre[b]), int(cu_q[b + 1] - cu_q[b])
+        vis = (L - Q) * Q + Q * (Q + 1) // 2
+        total += 4 * wl.D * wl.Hq * vis
+    return int(total)
+
+
 def _to_bf16_bits(x: np.ndarray) -> np.ndarray:
     import torch
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16) \
