@@ -509,6 +509,8 @@ def run_prefill(args, rank, world, local_rank):
     cu = torch.from_numpy(cu_q).to(dev_name)
     max_q = int(np.diff(cu_q).max())
     stream = torch.cuda.current_stream()
+    pkv.set_prefill_path(pkv.PKV_PREFILL_SINGLE_TILE if args.prefill_kernel == "single_tile"
+                         else pkv.PKV_PREFILL_AUTO)
 
     def step():
         pkv.paged_attention_prefill(out, q, dev["k_cache"], dev["v_cache"], bt, seq, cu, max_q,
@@ -540,7 +542,9 @@ def run_prefill(args, rank, world, local_rank):
                                    "Hq=32, Hkv=8, D=128, bs=16", "flops_per_step": flops},
             "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
-                         "traffic": None, "kernel": "paged_prefill_kernel", "peak_source": src},
+                         "traffic": None, "peak_source": src,
+                         "kernel": ("paged_prefill_kernel" if args.prefill_kernel == "single_tile"
+                                    else "paged_prefill_pp_kernel")},
             "gpu_launches": args.steps, "clocks": clocks.summary()}
 
 
@@ -588,6 +592,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
                     help="decode step (default) or multi-query chunked-append attention")
+    ap.add_argument("--prefill-kernel", choices=["two_tile", "single_tile"], default="two_tile",
+                    help="prefill kernel: warp-specialised two-tile (default) or single-tile")
     ap.add_argument("--path", choices=["auto", "cuda_cores", "tensor_cores"], default="auto",
                     help="decode kernel family (library default: auto)")
     ap.add_argument("--decode", choices=["auto", "plain", "shared_prefix"], default="auto",

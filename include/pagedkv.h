@@ -352,6 +352,18 @@ enum { PKV_PATH_AUTO = 0, PKV_PATH_CUDA_CORES = 1, PKV_PATH_TENSOR_CORES = 2 };
 int pkv_set_decode_path(int mode);
 
 /*
+ * Kernel used by paged_attention_prefill, set for the whole process (for
+ * testing and measuring both):
+ *   PKV_PREFILL_AUTO         D <= 128: the warp-specialised kernel with two
+ *                            query tiles per CTA; D = 256: one tile per CTA;
+ *   PKV_PREFILL_SINGLE_TILE  one query tile per CTA for every D.
+ * Both give results within the same bounds.  Returns the previous mode, or
+ * PKV_ERR_INVALID_ARG.
+ */
+enum { PKV_PREFILL_AUTO = 0, PKV_PREFILL_SINGLE_TILE = 1 };
+int pkv_set_prefill_path(int mode);
+
+/*
  * How paged_attention_decode with partition_size == 0 cuts the work, set for
  * the whole process:
  *   PKV_SPLIT_FIXED (default)  partitions of a library-chosen length, one CTA

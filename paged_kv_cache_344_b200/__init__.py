@@ -39,6 +39,8 @@ DEVERR_PREFIX = 0x20
 PKV_ERR_SCRATCH_LIMIT = -6
 PKV_SPLIT_FIXED = 0
 PKV_SPLIT_BALANCED = 1
+PKV_PREFILL_AUTO = 0
+PKV_PREFILL_SINGLE_TILE = 1
 NOALLOC_SCRATCH_BYTES = 16 << 20  # PKV_NOALLOC_SCRATCH_BYTES
 
 _lib = None
@@ -104,6 +106,8 @@ def lib() -> ctypes.CDLL:
     L.pkv_last_cuda_error.restype = i32
     L.pkv_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     L.pkv_device_errors.restype = i32
+    L.pkv_set_prefill_path.argtypes = [i32]
+    L.pkv_set_prefill_path.restype = i32
     L.pkv_set_decode_path.argtypes = [i32]
     L.pkv_set_decode_path.restype = i32
     L.pkv_set_decode_split.argtypes = [i32]
@@ -284,6 +288,13 @@ def set_decode_path(mode: int) -> int:
     """Select CUDA-core / tensor-core decode kernels process-wide; returns the old mode."""
     r = lib().pkv_set_decode_path(int(mode))
     _check("pkv_set_decode_path", min(r, 0))
+    return r
+
+
+def set_prefill_path(mode: int) -> int:
+    """Two-tile warp-specialised (auto) or single-tile prefill kernel; returns the old mode."""
+    r = lib().pkv_set_prefill_path(int(mode))
+    _check("pkv_set_prefill_path", min(r, 0))
     return r
 
 

@@ -22,6 +22,7 @@ thread_local int g_last_cuda_error = 0;
 std::atomic<int> g_decode_path{PKV_PATH_AUTO};
 std::atomic<int> g_decode_ctas{0};  // 0: as many as fit (at most 2 per SM)
 std::atomic<int> g_decode_split{PKV_SPLIT_FIXED};
+std::atomic<int> g_prefill_path{PKV_PREFILL_AUTO};
 
 constexpr int kSmCount = 148;  // B200
 
@@ -630,7 +631,10 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
   if ((int64_t)max_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
   if ((int64_t)max_seq_len > (int64_t)max_blocks * block_size) return PKV_ERR_OUT_OF_RANGE;
   const int TQ = pkv::kPrefillRows / G;
-  const int64_t q_tiles = ceil_div(max_q_len, TQ);
+  // Two query tiles per CTA on the warp-specialised kernel (D <= 128, which
+  // leaves TMEM room for both tiles' S and O); one on the single-tile kernel.
+  const bool two_tile = D <= 128 && g_prefill_path != PKV_PREFILL_SINGLE_TILE;
+  const int64_t q_tiles = ceil_div(max_q_len, two_tile ? 2 * TQ : TQ);
   if (B > 65535 || q_tiles > 65535) return PKV_ERR_OUT_OF_RANGE;
 
   pkv::PrefillParams p{};
@@ -669,17 +673,23 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
   if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
   if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
   dim3 grid((unsigned)Hkv, (unsigned)q_tiles, (unsigned)B);
-  auto launch = [&](auto kernel, size_t smem, std::atomic<uint64_t>& set) -> int {
+  auto launch = [&](auto kernel, size_t smem, std::atomic<uint64_t>& set, int threads) -> int {
     int rc2 = ensure_smem(kernel, smem, set);
     if (rc2 != PKV_OK) return rc2;
-    kernel<<<grid, pkv::kWarps * 32, smem, stream>>>(p, mq, mk, mv);
+    kernel<<<grid, threads, smem, stream>>>(p, mq, mk, mv);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? PKV_OK : cuda_fail(e);
   };
-  static std::atomic<uint64_t> set64{0}, set128{0}, set256{0};
-  if (D == 64) return launch(pkv::paged_prefill_kernel<64>, pkv::PrefillSmem<64>::kBytes, set64);
-  if (D == 128) return launch(pkv::paged_prefill_kernel<128>, pkv::PrefillSmem<128>::kBytes, set128);
-  return launch(pkv::paged_prefill_kernel<256>, pkv::PrefillSmem<256>::kBytes, set256);
+  static std::atomic<uint64_t> pp64{0}, pp128{0}, set64{0}, set128{0}, set256{0};
+  if (two_tile && D == 64)
+    return launch(pkv::paged_prefill_pp_kernel<64>, pkv::PpSmem<64>::kBytes, pp64, pkv::kPpThreads);
+  if (two_tile)
+    return launch(pkv::paged_prefill_pp_kernel<128>, pkv::PpSmem<128>::kBytes, pp128, pkv::kPpThreads);
+  const int th = pkv::kWarps * 32;
+  if (D == 64) return launch(pkv::paged_prefill_kernel<64>, pkv::PrefillSmem<64>::kBytes, set64, th);
+  if (D == 128)
+    return launch(pkv::paged_prefill_kernel<128>, pkv::PrefillSmem<128>::kBytes, set128, th);
+  return launch(pkv::paged_prefill_kernel<256>, pkv::PrefillSmem<256>::kBytes, set256, th);
 }
 
 int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int64_t P,
@@ -795,6 +805,11 @@ int pkv_set_decode_split(int mode) {
 int pkv_set_decode_ctas(int ctas) {
   if (ctas < 0) return PKV_ERR_INVALID_ARG;
   return g_decode_ctas.exchange(ctas);
+}
+
+int pkv_set_prefill_path(int mode) {
+  if (mode != PKV_PREFILL_AUTO && mode != PKV_PREFILL_SINGLE_TILE) return PKV_ERR_INVALID_ARG;
+  return g_prefill_path.exchange(mode);
 }
 
 int pkv_set_decode_path(int mode) {

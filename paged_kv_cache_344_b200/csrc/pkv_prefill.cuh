@@ -338,4 +338,389 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialised two-tile kernel (D = 64 or 128).
+//
+// One CTA owns two query tiles of 128 rows (tile 0 = query tokens i0 ..
+// i0 + TQ - 1, tile 1 = the next TQ) of one KV head, so every K/V tile brought
+// into shared memory serves 256 rows.  KV tiles are 128 tokens.  Roles:
+//  * warps 0-3 / 4-7: the softmax of tile 0 / tile 1 (thread = row);
+//  * warp 8: the producer (TMA: both query tiles, then K_0, V_0, K_1, ... into
+//    a ring of kRing slots, each one K or V tile);
+//  * warp 9: the MMA issuer (one lane) and TMEM owner.
+// TMEM (512 columns): S of tile t at 128 t, O of tile t at 256 + D t.  The
+// softmax of tile t reads S (fp32), writes P as bf16 pairs over the first 64
+// columns of the same S region, and the P V MMA takes P straight from TMEM.
+// MMA order per KV tile j:  P0 V_j, S0(j+1), P1 V_j, S1(j+1).  S_t(j+1)
+// overwrites the columns P_t(j) V_j reads, so the issuer waits for that P V to
+// complete first (while the other tile's MMA keeps the tensor pipe busy).  The
+// softmax of tile 0 thus overlaps P1 V_{j-1} and S1(j), and tile 1 overlaps
+// P0 V_j and S0(j+1).
+// The running maximum only moves when a tile's maximum exceeds it by more than
+// 2^8 (scores in log2 units), so O is rescaled rarely; P then stays below 256,
+// and the final O / l is the same quotient.
+// ---------------------------------------------------------------------------
+constexpr int kPpKv = 128;          // tokens per K/V tile (MMA N of S, K of P V)
+constexpr int kPpThreads = 320;     // 10 warps
+constexpr float kPpRescale = 8.0f;  // log2 growth of the row max that forces a rescale
+
+template <int D>
+struct PpSmem {
+  static constexpr int SUB = D / 64;
+  static constexpr int kRing = D == 64 ? 8 : 4;
+  static constexpr int kQTile = SUB * kPrefillRows * 128;  // one query tile
+  static constexpr int kKvTile = SUB * kPpKv * 128;        // one K or V tile
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = 2 * kQTile;
+  static constexpr int kOffBar = kOffRing + kRing * kKvTile;
+  // q_full, kv_full[kRing], kv_empty[kRing], s_full[2], p_full[2], o_full[2], done
+  static constexpr int kNumBars = 1 + 2 * kRing + 7;
+  static constexpr size_t kBytes = 1024 + (size_t)kOffBar + 8 * kNumBars;
+  static constexpr uint32_t kOCol = 256;
+  static constexpr uint32_t kCols = 512;
+};
+
+// Bounded wait that also gives up as soon as another role of the CTA has.
+__device__ __forceinline__ bool pp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      flag_error(PKV_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// The same, agreed by the whole warp (so that warp-collective instructions
+// after it are reached by all lanes or by none).
+__device__ __forceinline__ bool pp_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return __all_sync(kFull, pp_wait(bar, parity, abort));
+}
+
+// Row softmax of one 128-token S tile for the thread's row, P written back to
+// TMEM, O rescaled when the row max moved.
+template <int D>
+__device__ __forceinline__ void pp_softmax_tile(uint32_t s_tm, uint32_t o_tm, int j, int visible,
+                                                float cl2, bool pos, float& m_run, float& l_run) {
+  uint32_t s[4][32];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, s[c]);
+  tmem_wait_ld();
+  const int tbase = j * kPpKv;
+  float k = cl2;
+  float m_tile;
+  if (tbase + kPpKv > visible) {
+    // Diagonal (or fully masked) tile: scale first, then mask to -inf.
+    m_tile = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kPpKv; ++c) {
+      const float x = tbase + c < visible ? __uint_as_float(s[c / 32][c % 32]) * cl2 : -INFINITY;
+      s[c / 32][c % 32] = __float_as_uint(x);
+      m_tile = fmaxf(m_tile, x);
+    }
+    k = 1.f;
+  } else if (pos) {
+    float mx = __uint_as_float(s[0][0]);
+#pragma unroll
+    for (int c = 1; c < kPpKv; ++c) mx = fmaxf(mx, __uint_as_float(s[c / 32][c % 32]));
+    m_tile = mx * cl2;
+  } else {
+    float mn = __uint_as_float(s[0][0]);
+#pragma unroll
+    for (int c = 1; c < kPpKv; ++c) mn = fminf(mn, __uint_as_float(s[c / 32][c % 32]));
+    m_tile = mn * cl2;
+  }
+  float alpha = 1.f;
+  if (m_tile > m_run + kPpRescale) {  // also the first tile (m_run = -inf)
+    alpha = ex2_approx(m_run - m_tile);
+    m_run = m_tile;
+  }
+  const float neg_m = -m_run;
+  float sum = 0.f;
+  uint32_t pk[2][32];
+#pragma unroll
+  for (int c = 0; c < kPpKv; c += 2) {
+    const float p0 = ex2_approx(fmaf(__uint_as_float(s[c / 32][c % 32]), k, neg_m));
+    const float p1 = ex2_approx(fmaf(__uint_as_float(s[(c + 1) / 32][(c + 1) % 32]), k, neg_m));
+    sum += p0 + p1;
+    pk[c / 64][(c % 64) / 2] = pack_bf16x2(p0, p1);
+  }
+  l_run = l_run * alpha + sum;
+  if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t ov[32];
+      tmem_ld32(o_tm + cc * 32, ov);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+      tmem_st32(o_tm + cc * 32, ov);
+    }
+  }
+  tmem_st32(s_tm + 0, pk[0]);
+  tmem_st32(s_tm + 32, pk[1]);
+  tmem_wait_st();
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPpThreads, 1)
+    paged_prefill_pp_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV) {
+  using S = PpSmem<D>;
+  constexpr int R = S::kRing;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + R;
+  uint64_t* s_full = bars + 1 + 2 * R;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = s_full + 4;
+  uint64_t* done = s_full + 6;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+
+  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  const int kvh = blockIdx.x;
+  const int qt = gridDim.y - 1 - blockIdx.y;  // the longest tiles of a sequence first
+  const int b = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = p.G, TQ = p.TQ;
+  const int q0 = p.cu_q[b];
+  const int Q = p.cu_q[b + 1] - q0;
+  const int i0 = qt * 2 * TQ;
+  if (i0 >= Q) return;
+  int L = p.seq_lens[b];
+  const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
+  if (L > Lcap || Q > L) {
+    if (threadIdx.x == 0 && qt == 0 && kvh == 0) flag_error(PKV_DEVERR_SEQLEN);
+    if (Q > min(L, Lcap)) return;  // no consistent reading: rows are left unwritten
+    L = Lcap;
+  }
+  const int ctx = L - Q;
+  const int kv_end = ctx + min(Q, i0 + 2 * TQ);  // tokens any row of the CTA sees
+  const int n_kv = (kv_end + kPpKv - 1) / kPpKv;
+
+  if (warp == 9) {
+    tmem_alloc(&s_tmem, S::kCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(q_full, 1);
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+    }
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = s_tmem;
+  uint8_t* q_smem = smem + S::kOffQ;
+  uint8_t* ring = smem + S::kOffRing;
+
+  if (warp < 8) {
+    // ---- softmax of tile t = warp / 4; thread = row r ----
+    const int t = warp / 4;
+    const int r = threadIdx.x % 128;
+    const int i = i0 + t * TQ + r / G, g = r % G;
+    const bool row_valid = i < Q;
+    const int visible = min(ctx + i + 1, kv_end);
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t s_tm = tmem + 128u * t + lane_base;
+    const uint32_t o_tm = tmem + S::kOCol + (uint32_t)D * t + lane_base;
+    const float cl2 = p.scale_log2;
+    const bool pos = cl2 >= 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!(ok = pp_wait_warp(&s_full[t], (uint32_t)(j & 1), &s_abort))) break;
+      tc_fence_after_sync();
+      pp_softmax_tile<D>(s_tm, o_tm, j, visible, cl2, pos, m_run, l_run);
+      tc_fence_before_sync();
+      mbar_arrive(&p_full[t]);
+    }
+    if (ok) ok = pp_wait_warp(&o_full[t], (uint32_t)((n_kv - 1) & 1), &s_abort);
+    if (ok) {
+      tc_fence_after_sync();
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
+                            ((size_t)(q0 + i) * p.Hq + (size_t)kvh * G + g) * D;
+      const float inv = 1.f / l_run;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ov[32];
+        tmem_ld32(o_tm + cc * 32, ov);
+        tmem_wait_ld();
+        if (row_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ov[e + 0]) * inv, __uint_as_float(ov[e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ov[e + 4]) * inv, __uint_as_float(ov[e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ov[e + 6]) * inv, __uint_as_float(ov[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + cc * 32 + e) = w;
+          }
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // ---- producer ----
+    const uint64_t pol = l2_policy_evict_first();
+    const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks;
+    if (lane == 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      mbar_arrive_expect_tx(q_full, 2 * S::kQTile);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int sb = 0; sb < S::SUB; ++sb)
+          tma_load_3d(q_smem + t * S::kQTile + sb * (kPrefillRows * 128), &tmQ, q_full, sb * 64,
+                      kvh * G, q0 + i0 + t * TQ, pol);
+    }
+    int issued = 0;
+    int row = p.num_blocks * p.bs;  // box row of this lane's 16 tokens (past the end: zeros)
+    for (int idx = 0; idx < 2 * n_kv; ++idx) {
+      const int j = idx >> 1, slot = idx % R;
+      if ((idx & 1) == 0 && lane < kPpKv / kStageTokens) {
+        const int t0 = j * kPpKv + lane * kStageTokens;
+        row = p.num_blocks * p.bs;
+        if (t0 < kv_end) {
+          const int id = bt_row[t0 / p.bs];
+          if (id >= 0 && id < p.num_blocks) row = id * p.bs + t0 % p.bs;
+          else flag_error(PKV_DEVERR_BLOCK_ID);
+        }
+      }
+      if (!pp_wait_warp(&kv_empty[slot], (uint32_t)(((idx / R) & 1) ^ 1), &s_abort)) break;
+      if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], S::kKvTile);
+      __syncwarp();
+      if (lane < kPpKv / kStageTokens) {
+        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
+#pragma unroll
+        for (int sb = 0; sb < S::SUB; ++sb)
+          tma_load_3d(ring + slot * S::kKvTile + sb * (kPpKv * 128) + lane * (kStageTokens * 128),
+                      map, &kv_full[slot], sb * 64, kvh, row, pol);
+      }
+      issued = idx + 1;
+    }
+    // Loads still in flight after an abort land before the CTA lets go of its
+    // shared memory (bounded).
+    if (s_abort && lane == 0)
+      for (int idx = max(0, issued - R); idx < issued; ++idx)
+        mbar_wait_bounded(&kv_full[idx % R], (uint32_t)((idx / R) & 1));
+  } else {
+    // ---- MMA issuer ----
+    constexpr uint32_t kIdescS = umma_idesc_bf16(kPrefillRows, kPpKv, false);
+    constexpr uint32_t kIdescO = umma_idesc_bf16(kPrefillRows, D, true);
+    const bool leader = lane == 0;
+    const uint32_t q_addr = smem_u32(q_smem);
+    const uint32_t ring_addr = smem_u32(ring);
+    auto issue_s = [&](int t, int j) {
+      const uint32_t k_addr = ring_addr + (uint32_t)(((2 * j) % R) * S::kKvTile);
+      const uint32_t qa = q_addr + (uint32_t)(t * S::kQTile);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t ad = umma_desc_sw128(qa + (kk / 4) * (kPrefillRows * 128) + (kk % 4) * 32, 16, 1024);
+        const uint64_t bd = umma_desc_sw128(k_addr + (kk / 4) * (kPpKv * 128) + (kk % 4) * 32, 16, 1024);
+        umma_bf16(tmem + 128u * t, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&s_full[t]);
+    };
+    auto issue_pv = [&](int t, int j) {
+      const uint32_t v_addr = ring_addr + (uint32_t)(((2 * j + 1) % R) * S::kKvTile);
+#pragma unroll
+      for (int kk = 0; kk < kPpKv / 16; ++kk) {
+        const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, kPpKv * 128, 1024);
+        umma_bf16_tmem_a(tmem + S::kOCol + (uint32_t)D * t, tmem + 128u * t + 8u * kk, bd, kIdescO,
+                         (j > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&o_full[t]);
+    };
+    bool ok = pp_wait_warp(q_full, 0, &s_abort) && pp_wait_warp(&kv_full[0], 0, &s_abort);
+    if (ok) {
+      tc_fence_after_sync();
+      if (leader) {
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit(&kv_empty[0]);
+      }
+      __syncwarp();
+    }
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int iv = 2 * j + 1, ik = 2 * j + 2;
+      if (!(ok = pp_wait_warp(&kv_full[iv % R], (uint32_t)((iv / R) & 1), &s_abort))) break;
+      if (j == n_kv - 1 && kv_end < n_kv * kPpKv) {
+        // Tokens past the end: their V rows may hold anything (even NaN), and
+        // 0 * NaN must not reach O.
+        uint8_t* v_smem = ring + (iv % R) * S::kKvTile;
+        const int first = kv_end - j * kPpKv;
+        const int nvec = (kPpKv - first) * 8;
+        for (int sb = 0; sb < S::SUB; ++sb)
+          for (int v = lane; v < nvec; v += 32)
+            reinterpret_cast<uint4*>(v_smem + sb * (kPpKv * 128) + first * 128)[v] =
+                make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (!(ok = pp_wait_warp(&p_full[0], (uint32_t)(j & 1), &s_abort))) break;
+      tc_fence_after_sync();
+      if (leader) issue_pv(0, j);
+      __syncwarp();
+      if (j + 1 < n_kv) {
+        if (!(ok = pp_wait_warp(&kv_full[ik % R], (uint32_t)((ik / R) & 1), &s_abort))) break;
+        if (!(ok = pp_wait_warp(&o_full[0], (uint32_t)(j & 1), &s_abort))) break;
+        tc_fence_after_sync();
+        if (leader) issue_s(0, j + 1);
+        __syncwarp();
+      }
+      if (!(ok = pp_wait_warp(&p_full[1], (uint32_t)(j & 1), &s_abort))) break;
+      tc_fence_after_sync();
+      if (leader) {
+        issue_pv(1, j);
+        umma_commit(&kv_empty[iv % R]);
+      }
+      __syncwarp();
+      if (j + 1 < n_kv) {
+        if (!(ok = pp_wait_warp(&o_full[1], (uint32_t)(j & 1), &s_abort))) break;
+        tc_fence_after_sync();
+        if (leader) {
+          issue_s(1, j + 1);
+          umma_commit(&kv_empty[ik % R]);
+        }
+        __syncwarp();
+      }
+    }
+    // Every MMA issued has finished before TMEM is released (bounded).
+    if (leader) {
+      umma_commit(done);
+      mbar_wait_bounded(done, 0);
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, S::kCols);
+  }
+}
+
 }  // namespace pkv

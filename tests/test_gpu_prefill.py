@@ -1,8 +1,10 @@
 """GPU parity of the tcgen05 multi-query (prefill / chunked append) attention against the
 oracle's fp64 definition: every query row is causal attention over the tokens up to its
 own position.  Covers pure prefill (no context), chunks appended to long contexts, single
-queries, query tiles cut mid-sequence, G = 1..16, D = 64/128/256, block sizes 16 and 32,
-and NaN-poisoned unused slots."""
+queries, query tiles cut mid-sequence, G = 1..16, D = 64/128/256, block sizes 16 to 256,
+NaN-poisoned unused slots, positive, negative and zero scales and score ranges that move
+the running maximum many times; on both kernels (two query tiles per CTA, warp-specialised,
+and one tile per CTA)."""
 import numpy as np
 import pytest
 import torch
@@ -15,7 +17,7 @@ from gpu_util import assert_attention_close, to_device, widen
 pytestmark = pytest.mark.gpu
 
 
-def _run(Hq, Hkv, D, bs, lens, qlens, seed=3):
+def _run(Hq, Hkv, D, bs, lens, qlens, seed=3, scale=None):
     wl = workloads.custom("pf", "bf16", len(lens), Hq, Hkv, D, bs, lens, seed=seed)
     host = workloads.host_tensors(wl)
     rng = np.random.default_rng(seed + 1)
@@ -24,24 +26,28 @@ def _run(Hq, Hkv, D, bs, lens, qlens, seed=3):
     q = torch.from_numpy(qf).to(torch.bfloat16)
     q_bits = q.view(torch.int16).numpy().view(np.uint16)
     seq = np.asarray(lens, np.int32)
+    scale = wl.scale if scale is None else scale
     ref = oracle.paged_prefill(q_bits, host["k_cache"], host["v_cache"], wl.block_tables, seq, cu,
-                               wl.scale)
+                               scale)
     dev_q = q.cuda()
     out = torch.full_like(dev_q, float("nan"))
     pkv.paged_attention_prefill(out, dev_q, to_device(host["k_cache"], "bf16"),
                                 to_device(host["v_cache"], "bf16"),
                                 torch.from_numpy(wl.block_tables).cuda(),
                                 torch.from_numpy(seq).cuda(), torch.from_numpy(cu).cuda(),
-                                int(max(qlens)), int(seq.max()), wl.scale)
+                                int(max(qlens)), int(seq.max()), scale)
     torch.cuda.synchronize()
     return widen(out), ref
 
 
-@pytest.fixture(autouse=True)
-def _clean():
+@pytest.fixture(autouse=True, params=["auto", "single_tile"])
+def path(request):
+    old = pkv.set_prefill_path(pkv.PKV_PREFILL_AUTO if request.param == "auto"
+                               else pkv.PKV_PREFILL_SINGLE_TILE)
     pkv.device_errors(clear=True)
-    yield
+    yield request.param
     torch.cuda.synchronize()
+    pkv.set_prefill_path(old)
     assert pkv.device_errors() == 0
 
 
@@ -81,3 +87,34 @@ def test_prefill_single_query_equals_decode():
     ref = oracle.paged_decode(host["q"], host["k_cache"], host["v_cache"], wl.block_tables,
                               np.asarray(lens, np.int32), wl.scale)
     assert_attention_close(widen(out_p), ref, "bf16", "prefill Q=1")
+
+
+@pytest.mark.parametrize("qlens", [[31, 32, 33, 63, 64, 65, 96, 128, 129]],
+                         ids=["around-two-tiles"])
+def test_prefill_two_tile_edges(qlens):
+    """G = 4 (32 query tokens per 128-row tile): chunks that end inside the first tile,
+    exactly on the tile pair, and one past it; contexts of 0 and 100 tokens."""
+    lens = [q + (0 if i % 2 else 100) for i, q in enumerate(qlens)]
+    got, ref = _run(32, 8, 128, 16, lens, qlens, seed=11)
+    assert_attention_close(got, ref, "bf16", "two-tile edges")
+
+
+def test_prefill_long_context_ring_wrap():
+    """Chunks appended to 3000-4700 cached tokens: dozens of K/V tiles cycle the ring."""
+    got, ref = _run(32, 8, 128, 16, [3000, 4700, 2100], [300, 512, 77], seed=13)
+    assert_attention_close(got, ref, "bf16", "long context")
+
+
+@pytest.mark.parametrize("bs", [64, 128, 256])
+def test_prefill_large_blocks(bs):
+    got, ref = _run(16, 2, 128, bs, [900, 260, 1], [150, 260, 1], seed=15)
+    assert_attention_close(got, ref, "bf16", f"bs={bs}")
+
+
+@pytest.mark.parametrize("scale", [1.0, -0.3, 0.0], ids=["wide", "negative", "zero"])
+def test_prefill_scales(scale):
+    """scale 1.0 spreads the scores over hundreds of log2 units (the running maximum moves
+    often and O is rescaled); a negative scale flips which score is largest; zero gives
+    uniform weights over the visible prefix."""
+    got, ref = _run(16, 4, 128, 16, [700, 130, 64], [200, 130, 5], seed=17, scale=scale)
+    assert_attention_close(got, ref, "bf16", f"scale={scale}")
