@@ -511,10 +511,14 @@ def run_prefill(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     pkv.set_prefill_path(pkv.PKV_PREFILL_SINGLE_TILE if args.prefill_kernel == "single_tile"
                          else pkv.PKV_PREFILL_AUTO)
+    ws = None
+    if args.prefill_kernel == "two_tile":  # persistent, longest-first schedule
+        n = pkv.paged_attention_prefill_workspace_size(wl.B, wl.Hq, wl.Hkv, int(np.diff(cu_q).max()))
+        ws = torch.empty(n, dtype=torch.uint8, device=dev_name)
 
     def step():
         pkv.paged_attention_prefill(out, q, dev["k_cache"], dev["v_cache"], bt, seq, cu, max_q,
-                                    int(wl.seq_lens_pre.max()), wl.scale)
+                                    int(wl.seq_lens_pre.max()), wl.scale, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -544,7 +548,8 @@ def run_prefill(args, rank, world, local_rank):
                          "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
                          "traffic": None, "peak_source": src,
                          "kernel": ("paged_prefill_kernel" if args.prefill_kernel == "single_tile"
-                                    else "paged_prefill_pp_kernel")},
+                                    else "paged_prefill_pp_kernel"),
+                         "schedule": args.prefill_kernel},
             "gpu_launches": args.steps, "clocks": clocks.summary()}
 
 
@@ -592,8 +597,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
                     help="decode step (default) or multi-query chunked-append attention")
-    ap.add_argument("--prefill-kernel", choices=["two_tile", "single_tile"], default="two_tile",
-                    help="prefill kernel: warp-specialised two-tile (default) or single-tile")
+    ap.add_argument("--prefill-kernel", choices=["two_tile", "per_item", "single_tile"],
+                    default="two_tile",
+                    help="prefill kernel: warp-specialised two-tile, persistent with the "
+                         "longest-first schedule (default); the same, one CTA per item; or "
+                         "single-tile")
     ap.add_argument("--path", choices=["auto", "cuda_cores", "tensor_cores"], default="auto",
                     help="decode kernel family (library default: auto)")
     ap.add_argument("--decode", choices=["auto", "plain", "shared_prefix"], default="auto",

@@ -172,17 +172,28 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
  *   out, q        device [total_q][Hq][D]
  *   cu_q          device [B + 1] int32, non-decreasing, cu_q[B] = total_q
  *   max_q_len     host upper bound of Q; max_seq_len host upper bound of L
- * It runs on the tcgen05 tensor cores.  Each CTA takes 128 query rows (128/G
- * tokens x G heads of one KV head) and streams the sequence's K/V in 64-token
- * tiles through TMEM accumulators.  bf16 only; G in {1, 2, 4, 8, 16}; D in
- * {64, 128, 256}; block_size a multiple of 16 up to 256.  A sequence with Q > L
- * flags PKV_DEVERR_SEQLEN and its rows are not written.
+ * It runs on the tcgen05 tensor cores: a query tile is 128 rows (128/G tokens x
+ * the G query heads of one KV head); S = Q K^T and O += P V accumulate in tensor
+ * memory.  For D <= 128 a CTA takes two query tiles of one KV head and streams
+ * the sequence's K/V in 128-token tiles (the two tiles' softmaxes alternate
+ * with the other tile's MMAs); for D = 256 one tile and 64-token K/V tiles.
+ * bf16 only; G in {1, 2, 4, 8, 16}; D in {64, 128, 256}; block_size a multiple
+ * of 16 up to 256.  A sequence with Q > L flags PKV_DEVERR_SEQLEN and its rows
+ * are not written.
+ *   workspace     device scratch of paged_attention_prefill_workspace_size()
+ *                 bytes (4-byte aligned, no initialisation needed) or NULL.
+ *                 With it (D <= 128), a first small kernel orders the work
+ *                 items (pairs of query tiles) longest first and one CTA per
+ *                 SM takes them in that order; without it, one CTA per item.
+ *                 A workspace serves one call at a time (stream order).
  */
+size_t paged_attention_prefill_workspace_size(int B, int Hq, int Hkv, int max_q_len);
 int paged_attention_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                             const int32_t *block_tables, int max_blocks, const int32_t *seq_lens,
                             const int32_t *cu_q, int total_q, int max_q_len, int max_seq_len,
                             int B, int Hq, int Hkv, int D, int block_size, int64_t num_blocks,
-                            float scale, pkv_dtype dtype, pkv_stream_t stream);
+                            float scale, pkv_dtype dtype, void *workspace,
+                            size_t workspace_bytes, pkv_stream_t stream);
 
 /*
  * paged_decode_step: one whole decode step in one launch.  For every sequence b

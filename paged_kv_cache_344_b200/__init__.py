@@ -80,8 +80,10 @@ def lib() -> ctypes.CDLL:
     L.paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
                                          i32, i64, f32, i32, i32, vp, sz, vp]
     L.paged_attention_decode.restype = i32
+    L.paged_attention_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
+    L.paged_attention_prefill_workspace_size.restype = sz
     L.paged_attention_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
-                                          i32, i32, i32, i32, i64, f32, i32, vp]
+                                          i32, i32, i32, i32, i64, f32, i32, vp, sz, vp]
     L.paged_attention_prefill.restype = i32
     L.paged_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
                                     i32, i32, i64, f32, i32, i32, vp, sz, vp]
@@ -187,16 +189,25 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, max
         _stream(q, stream)))
 
 
+def paged_attention_prefill_workspace_size(B, Hq, Hkv, max_q_len) -> int:
+    """Bytes of the scratch that lets paged_attention_prefill schedule its work longest first."""
+    return int(lib().paged_attention_prefill_workspace_size(B, Hq, Hkv, int(max_q_len)))
+
+
 def paged_attention_prefill(out, q, k_cache, v_cache, block_tables, seq_lens, cu_q, max_q_len,
-                            max_seq_len, scale, stream=None) -> None:
+                            max_seq_len, scale, workspace=None, stream=None) -> None:
     """Causal multi-query attention: rows ``cu_q[b] .. cu_q[b+1]-1`` of ``q [T,Hq,D]`` are the
-    last queries of sequence b (tcgen05 tensor cores)."""
+    last queries of sequence b (tcgen05 tensor cores).  ``workspace`` (a device tensor of at
+    least ``paged_attention_prefill_workspace_size`` bytes, or None) enables the persistent,
+    longest-first schedule."""
     T, Hq, D = q.shape
     NB, bs, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("paged_attention_prefill", lib().paged_attention_prefill(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         block_tables.shape[1], _ptr(seq_lens), _ptr(cu_q), T, int(max_q_len), int(max_seq_len),
-        seq_lens.shape[0], Hq, Hkv, D, bs, NB, float(scale), _dtype_code(q), _stream(q, stream)))
+        seq_lens.shape[0], Hq, Hkv, D, bs, NB, float(scale), _dtype_code(q), _ptr(workspace),
+        ws_bytes, _stream(q, stream)))
 
 
 def paged_decode_step(out, q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens,

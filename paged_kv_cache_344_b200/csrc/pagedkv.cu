@@ -26,6 +26,21 @@ std::atomic<int> g_prefill_path{PKV_PREFILL_AUTO};
 
 constexpr int kSmCount = 148;  // B200
 
+// Multiprocessors of the current device (looked up once per device).
+cudaError_t sm_count(int* out) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && cache[dev].load() > 0) {
+    *out = cache[dev].load();
+    return cudaSuccess;
+  }
+  e = cudaDeviceGetAttribute(out, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev].store(*out);
+  return e;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
@@ -604,11 +619,22 @@ int paged_decode_step_shared_prefix(void* out, const void* q, const void* k_new,
                      workspace_bytes, stream, step);
 }
 
+size_t paged_attention_prefill_workspace_size(int B, int Hq, int Hkv, int max_q_len) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_q_len <= 0 || Hq % Hkv != 0) return 0;
+  const int G = Hq / Hkv;
+  if (G > pkv::kPrefillRows) return 0;
+  const int64_t nqt = ceil_div(max_q_len, 2 * (pkv::kPrefillRows / G));
+  const int64_t items = (int64_t)B * nqt * Hkv;
+  if (items > 0x7fffffffLL) return 0;
+  return (size_t)(2 + items) * sizeof(int32_t);
+}
+
 int paged_attention_prefill(void* out, const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
                             const int32_t* cu_q, int total_q, int max_q_len, int max_seq_len,
                             int B, int Hq, int Hkv, int D, int block_size, int64_t num_blocks,
-                            float scale, pkv_dtype dtype, pkv_stream_t stream) {
+                            float scale, pkv_dtype dtype, void* workspace,
+                            size_t workspace_bytes, pkv_stream_t stream) {
   if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
   if (B < 0 || total_q < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 ||
       max_blocks <= 0 || num_blocks <= 0 || max_seq_len < 0 || max_q_len < 0 ||
@@ -636,6 +662,11 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
   const bool two_tile = D <= 128 && g_prefill_path != PKV_PREFILL_SINGLE_TILE;
   const int64_t q_tiles = ceil_div(max_q_len, two_tile ? 2 * TQ : TQ);
   if (B > 65535 || q_tiles > 65535) return PKV_ERR_OUT_OF_RANGE;
+  if (workspace) {
+    if ((reinterpret_cast<uintptr_t>(workspace) & 3u) ||
+        workspace_bytes < paged_attention_prefill_workspace_size(B, Hq, Hkv, max_q_len))
+      return PKV_ERR_INVALID_ARG;
+  }
 
   pkv::PrefillParams p{};
   p.out = out;
@@ -651,6 +682,9 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
   p.bs = block_size;
   p.num_blocks = (int)num_blocks;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.nqt = (int)q_tiles;
+  p.n_items = (int)((int64_t)B * q_tiles * Hkv);
+  p.sched = nullptr;
 
   // Query rows [T][Hq][D] as a 3-D tensor {D, Hq, T}; one box = 128 rows of one
   // KV head: {64, G, 128 / G}, 128-byte swizzled (the K-major MMA operand).
@@ -681,10 +715,22 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
     return e == cudaSuccess ? PKV_OK : cuda_fail(e);
   };
   static std::atomic<uint64_t> pp64{0}, pp128{0}, set64{0}, set128{0}, set256{0};
-  if (two_tile && D == 64)
-    return launch(pkv::paged_prefill_pp_kernel<64>, pkv::PpSmem<64>::kBytes, pp64, pkv::kPpThreads);
-  if (two_tile)
+  if (two_tile) {
+    // With a workspace: order the items longest first, then one persistent CTA
+    // per SM takes them in that order.  Without: one CTA per item.
+    if (workspace) {
+      p.sched = static_cast<int*>(workspace);
+      pkv::prefill_schedule_kernel<<<1, pkv::kSchedThreads, 0, stream>>>(p);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return cuda_fail(e);
+      int sms = 0;
+      if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e);
+      grid = dim3((unsigned)std::min<int64_t>(sms, p.n_items), 1, 1);
+    }
+    if (D == 64)
+      return launch(pkv::paged_prefill_pp_kernel<64>, pkv::PpSmem<64>::kBytes, pp64, pkv::kPpThreads);
     return launch(pkv::paged_prefill_pp_kernel<128>, pkv::PpSmem<128>::kBytes, pp128, pkv::kPpThreads);
+  }
   const int th = pkv::kWarps * 32;
   if (D == 64) return launch(pkv::paged_prefill_kernel<64>, pkv::PrefillSmem<64>::kBytes, set64, th);
   if (D == 128)

@@ -46,6 +46,12 @@ struct PrefillParams {
   int bs;
   int num_blocks;
   float scale_log2;
+  // Two-tile kernel: work item = ((b * nqt + qt) * Hkv + kvh), one pair of
+  // query tiles of one KV head.  sched (or NULL) = {next item, items with
+  // work, order[...] longest first} for the persistent launch.
+  int nqt;
+  int n_items;
+  int* sched;
 };
 
 template <int D>
@@ -343,26 +349,34 @@ __global__ void __launch_bounds__(kWarps * 32)
 //
 // One CTA owns two query tiles of 128 rows (tile 0 = query tokens i0 ..
 // i0 + TQ - 1, tile 1 = the next TQ) of one KV head, so every K/V tile brought
-// into shared memory serves 256 rows.  KV tiles are 128 tokens.  Roles:
+// into shared memory serves 256 rows.  Roles:
 //  * warps 0-3 / 4-7: the softmax of tile 0 / tile 1 (thread = row);
 //  * warp 8: the producer (TMA: both query tiles, then K_0, V_0, K_1, ... into
 //    a ring of kRing slots, each one K or V tile);
-//  * warp 9: the MMA issuer (one lane) and TMEM owner.
-// TMEM (512 columns): S of tile t at 128 t, O of tile t at 256 + D t.  The
-// softmax of tile t reads S (fp32), writes P as bf16 pairs over the first 64
-// columns of the same S region, and the P V MMA takes P straight from TMEM.
-// MMA order per KV tile j:  P0 V_j, S0(j+1), P1 V_j, S1(j+1).  S_t(j+1)
-// overwrites the columns P_t(j) V_j reads, so the issuer waits for that P V to
-// complete first (while the other tile's MMA keeps the tensor pipe busy).  The
-// softmax of tile 0 thus overlaps P1 V_{j-1} and S1(j), and tile 1 overlaps
-// P0 V_j and S0(j+1).
+//  * warp 9: the MMA issuer (one lane) and TMEM owner; warps 10-11 idle.
+// The three warpgroups launch with 168 registers a thread; the third gives up
+// all but kPpRegsIo and the two softmax warpgroups take kPpRegsSoftmax
+// (2 x 128 x 200 + 128 x 96 <= 384 x 168).
+//
+// K/V tiles are 128 tokens.  TMEM (512 columns): S of tile t at 128 t, O of
+// tile t at 256 + D t.  The softmax of tile t reads S (fp32), writes P as bf16
+// pairs over the first 64 columns of the same S region, and the P V MMA takes
+// P straight from TMEM.  MMA order per KV tile j:  P0 V_j, S0(j+1), P1 V_j,
+// S1(j+1).  S_t(j+1) overwrites the columns P_t(j) V_j reads, so the issuer
+// waits for that P V to complete first (while the other tile's MMA keeps the
+// tensor pipe busy).  The softmax of tile 0 thus overlaps P1 V_{j-1} and
+// S1(j), and tile 1 overlaps P0 V_j and S0(j+1).
 // The running maximum only moves when a tile's maximum exceeds it by more than
 // 2^8 (scores in log2 units), so O is rescaled rarely; P then stays below 256,
 // and the final O / l is the same quotient.
 // ---------------------------------------------------------------------------
 constexpr int kPpKv = 128;          // tokens per K/V tile (MMA N of S, K of P V)
-constexpr int kPpThreads = 320;     // 10 warps
+constexpr int kPpThreads = 384;     // 3 warpgroups
 constexpr float kPpRescale = 8.0f;  // log2 growth of the row max that forces a rescale
+constexpr uint32_t kPpRegsSoftmax = 200;
+constexpr uint32_t kPpRegsIo = 96;
+static_assert(2 * 128 * kPpRegsSoftmax + 128 * kPpRegsIo <= kPpThreads * 168,
+              "register split exceeds the launch allocation");
 
 template <int D>
 struct PpSmem {
@@ -370,24 +384,27 @@ struct PpSmem {
   static constexpr int kRing = D == 64 ? 8 : 4;
   static constexpr int kQTile = SUB * kPrefillRows * 128;  // one query tile
   static constexpr int kKvTile = SUB * kPpKv * 128;        // one K or V tile
+  static_assert(kKvTile % 1024 == 0, "ring slots keep the 1024-byte swizzle alignment");
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = 2 * kQTile;
   static constexpr int kOffBar = kOffRing + kRing * kKvTile;
-  // q_full, kv_full[kRing], kv_empty[kRing], s_full[2], p_full[2], o_full[2], done
-  static constexpr int kNumBars = 1 + 2 * kRing + 7;
+  // q_full, q_empty, kv_full[kRing], kv_empty[kRing], s_full[2], p_full[2],
+  // o_full[2], item_full[2], item_empty[2], done
+  static constexpr int kNumBars = 2 + 2 * kRing + 11;
   static constexpr size_t kBytes = 1024 + (size_t)kOffBar + 8 * kNumBars;
-  static constexpr uint32_t kOCol = 256;
+  static_assert(kBytes <= 227 * 1024, "shared memory");
+  static constexpr uint32_t kSCol = 0, kOCol = 256;  // + 128 t, + D t; P over S
   static constexpr uint32_t kCols = 512;
 };
 
 // Bounded wait that also gives up as soon as another role of the CTA has.
 __device__ __forceinline__ bool pp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_timer_ns();
+  const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (clock64() - t0 > kWaitLimitCycles) {
       *abort = 1;
       flag_error(PKV_DEVERR_TIMEOUT);
       return false;
@@ -401,55 +418,115 @@ __device__ __forceinline__ bool pp_wait_warp(uint64_t* bar, uint32_t parity, vol
   return __all_sync(kFull, pp_wait(bar, parity, abort));
 }
 
-// Row softmax of one 128-token S tile for the thread's row, P written back to
-// TMEM, O rescaled when the row max moved.
+// Arrive once for the warp, after its tensor-memory accesses are complete.
+__device__ __forceinline__ void pp_warp_arrive(uint64_t* bar) {
+  tc_fence_before_sync();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// 2^x for a pair, on the FMA pipe instead of the special-function unit:
+// x = n + f with n = round(x) (the 1.5 * 2^23 addition leaves n in the low
+// mantissa bits of t) and f in [-1/2, 1/2]; 2^f is a cubic, fitted here
+// (minimax over [-1/2, 1/2], relative error 7.5e-5, below bf16's 2^-9); 2^n is
+// added to its exponent field.  x is clamped at -126 (2^-126 is zero at the
+// precision P keeps); NaN stays NaN.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  x.x = x.x < -126.f ? -126.f : x.x;
+  x.y = x.y < -126.f ? -126.f : x.y;
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = ffma2(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.242611125f, 0.242611125f));
+  q = ffma2(q, f, make_float2(0.693260968f, 0.693260968f));
+  q = ffma2(q, f, make_float2(0.999928057f, 0.999928057f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Of every 8 pairs of probabilities, kPpPolyPairs take exp2_poly2 (the rest
+// the special-function unit).
+#ifndef PKV_PP_POLY_PAIRS
+#define PKV_PP_POLY_PAIRS 0
+#endif
+constexpr int kPpPolyPairs = PKV_PP_POLY_PAIRS;
+
+// One K/V tile of the row softmax for the thread's row: read S_t(j), compute P
+// and the running max / sum, rescale O if the max moved (the issuer computed
+// S_t(j) only after P_t(j-1) V_{j-1} was done, so O is final), and write P
+// over S.
 template <int D>
 __device__ __forceinline__ void pp_softmax_tile(uint32_t s_tm, uint32_t o_tm, int j, int visible,
                                                 float cl2, bool pos, float& m_run, float& l_run) {
-  uint32_t s[4][32];
+  uint32_t sv[4][32];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, s[c]);
+  for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + c * 32, sv[c]);
   tmem_wait_ld();
+  float x[kPpKv];
+#pragma unroll
+  for (int c = 0; c < kPpKv; ++c) x[c] = __uint_as_float(sv[c / 32][c % 32]);
   const int tbase = j * kPpKv;
-  float k = cl2;
-  float m_tile;
-  if (tbase + kPpKv > visible) {
+  // Reductions run over kAcc independent partial results (a tree, not a chain).
+  constexpr int kAcc = 8;
+  const bool masked = tbase + kPpKv > visible;
+  const bool take_max = masked || pos;  // masked scores are already scaled
+  const float k = masked ? 1.f : cl2;   // multiplier of x in the exponent
+  if (masked) {
     // Diagonal (or fully masked) tile: scale first, then mask to -inf.
-    m_tile = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kPpKv; ++c) {
-      const float x = tbase + c < visible ? __uint_as_float(s[c / 32][c % 32]) * cl2 : -INFINITY;
-      s[c / 32][c % 32] = __float_as_uint(x);
-      m_tile = fmaxf(m_tile, x);
-    }
-    k = 1.f;
-  } else if (pos) {
-    float mx = __uint_as_float(s[0][0]);
-#pragma unroll
-    for (int c = 1; c < kPpKv; ++c) mx = fmaxf(mx, __uint_as_float(s[c / 32][c % 32]));
-    m_tile = mx * cl2;
-  } else {
-    float mn = __uint_as_float(s[0][0]);
-#pragma unroll
-    for (int c = 1; c < kPpKv; ++c) mn = fminf(mn, __uint_as_float(s[c / 32][c % 32]));
-    m_tile = mn * cl2;
+    for (int c = 0; c < kPpKv; ++c) x[c] = tbase + c < visible ? x[c] * cl2 : -INFINITY;
   }
+  float part[kAcc];
+#pragma unroll
+  for (int a = 0; a < kAcc; ++a) part[a] = x[a];
+  if (take_max) {
+#pragma unroll
+    for (int c = kAcc; c < kPpKv; c += 2 * kAcc)
+#pragma unroll
+      for (int a = 0; a < kAcc; ++a)
+        part[a] = fmax3(part[a], x[c + a], x[c + kAcc + a < kPpKv ? c + kAcc + a : c + a]);
+  } else {
+#pragma unroll
+    for (int c = kAcc; c < kPpKv; c += 2 * kAcc)
+#pragma unroll
+      for (int a = 0; a < kAcc; ++a)
+        part[a] = fmin3(part[a], x[c + a], x[c + kAcc + a < kPpKv ? c + kAcc + a : c + a]);
+  }
+#pragma unroll
+  for (int w = kAcc / 2; w > 0; w /= 2)
+#pragma unroll
+    for (int a = 0; a < w; ++a)
+      part[a] = take_max ? fmaxf(part[a], part[a + w]) : fminf(part[a], part[a + w]);
+  const float m_tile = masked ? part[0] : part[0] * k;
   float alpha = 1.f;
   if (m_tile > m_run + kPpRescale) {  // also the first tile (m_run = -inf)
     alpha = ex2_approx(m_run - m_tile);
     m_run = m_tile;
   }
-  const float neg_m = -m_run;
-  float sum = 0.f;
+  const float2 kk2 = make_float2(k, k), nm2 = make_float2(-m_run, -m_run);
+  float2 acc[kAcc / 2];
+#pragma unroll
+  for (int a = 0; a < kAcc / 2; ++a) acc[a] = make_float2(0.f, 0.f);
   uint32_t pk[2][32];
 #pragma unroll
   for (int c = 0; c < kPpKv; c += 2) {
-    const float p0 = ex2_approx(fmaf(__uint_as_float(s[c / 32][c % 32]), k, neg_m));
-    const float p1 = ex2_approx(fmaf(__uint_as_float(s[(c + 1) / 32][(c + 1) % 32]), k, neg_m));
-    sum += p0 + p1;
-    pk[c / 64][(c % 64) / 2] = pack_bf16x2(p0, p1);
+    const float2 e = ffma2(make_float2(x[c], x[c + 1]), kk2, nm2);
+    float2 pr;
+    if ((c / 2) % 8 < kPpPolyPairs) {
+      pr = exp2_poly2(e);
+    } else {
+      pr.x = ex2_approx(e.x);
+      pr.y = ex2_approx(e.y);
+    }
+    acc[(c / 2) % (kAcc / 2)] = fadd2(acc[(c / 2) % (kAcc / 2)], pr);
+    pk[c / 64][(c % 64) / 2] = pack_bf16x2(pr.x, pr.y);
   }
-  l_run = l_run * alpha + sum;
+#pragma unroll
+  for (int w = kAcc / 4; w > 0; w /= 2)
+#pragma unroll
+    for (int a = 0; a < w; ++a) acc[a] = fadd2(acc[a], acc[a + w]);
+  l_run = l_run * alpha + (acc[0].x + acc[0].y);
   if (j > 0 && __any_sync(kFull, alpha != 1.f)) {
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -466,6 +543,99 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_tm, uint32_t o_tm, in
   tmem_wait_st();
 }
 
+// One work item of the two-tile kernel: which rows, which tokens they see.
+struct PpItem {
+  int b, kvh, q0, Q, i0, ctx, kv_end, n_kv;  // n_kv = 0: nothing to do
+  bool bad_len;                              // L > the table's capacity or Q > L
+};
+
+__device__ __forceinline__ PpItem pp_item(const PrefillParams& p, int item) {
+  PpItem it{};
+  it.kvh = item % p.Hkv;
+  const int r = item / p.Hkv;
+  const int qt = r % p.nqt;
+  it.b = r / p.nqt;
+  it.q0 = p.cu_q[it.b];
+  it.Q = p.cu_q[it.b + 1] - it.q0;
+  it.i0 = qt * 2 * p.TQ;
+  it.n_kv = 0;
+  int L = p.seq_lens[it.b];
+  const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
+  it.bad_len = L > Lcap || it.Q > L;
+  if (it.i0 >= it.Q || it.Q > min(L, Lcap)) return it;  // no rows, or no consistent reading
+  L = min(L, Lcap);
+  it.ctx = L - it.Q;
+  it.kv_end = it.ctx + min(it.Q, it.i0 + 2 * p.TQ);  // tokens any row of the item sees
+  it.n_kv = (it.kv_end + kPpKv - 1) / kPpKv;
+  return it;
+}
+
+// Orders the work items longest first (a counting sort on the number of K/V
+// tiles, one block of kSchedThreads threads), for the persistent launch, which
+// takes them in that order from an atomic counter: the longest items start
+// first and the short ones fill the tail.  Also flags bad lengths.
+constexpr int kSchedThreads = 1024;  // = number of buckets
+
+__global__ void __launch_bounds__(kSchedThreads)
+    prefill_schedule_kernel(const PrefillParams p) {
+  __shared__ int hist[kSchedThreads];
+  __shared__ int warp_sum[kSchedThreads / 32];
+  __shared__ int n_work;
+  const int tid = threadIdx.x;
+  hist[tid] = 0;
+  if (tid == 0) n_work = 0;
+  __syncthreads();
+  // bucket kSchedThreads - 1 - min(n_kv, kSchedThreads - 1): thread order is then
+  // descending cost
+  for (int item = tid; item < p.n_items; item += kSchedThreads) {
+    const PpItem it = pp_item(p, item);
+    if (it.bad_len && it.i0 == 0 && it.kvh == 0) flag_error(PKV_DEVERR_SEQLEN);
+    if (it.n_kv > 0) {
+      atomicAdd(&hist[kSchedThreads - 1 - min(it.n_kv, kSchedThreads - 1)], 1);
+      atomicAdd(&n_work, 1);
+    }
+  }
+  __syncthreads();
+  // Exclusive scan of hist in thread order.
+  const int v = hist[tid];
+  int incl = v;
+#pragma unroll
+  for (int d = 1; d < 32; d *= 2) {
+    const int y = __shfl_up_sync(kFull, incl, d);
+    if ((tid & 31) >= d) incl += y;
+  }
+  if ((tid & 31) == 31) warp_sum[tid / 32] = incl;
+  __syncthreads();
+  if (tid < 32) {
+    int w = warp_sum[tid];
+#pragma unroll
+    for (int d = 1; d < 32; d *= 2) {
+      const int y = __shfl_up_sync(kFull, w, d);
+      if (tid >= d) w += y;
+    }
+    warp_sum[tid] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  hist[tid] = incl - v + (tid >= 32 ? warp_sum[tid / 32 - 1] : 0);
+  __syncthreads();
+  int* order = p.sched + 2;
+  for (int item = tid; item < p.n_items; item += kSchedThreads) {
+    const PpItem it = pp_item(p, item);
+    if (it.n_kv > 0)
+      order[atomicAdd(&hist[kSchedThreads - 1 - min(it.n_kv, kSchedThreads - 1)], 1)] = item;
+  }
+  if (tid == 0) {
+    p.sched[0] = 0;
+    p.sched[1] = n_work;
+  }
+}
+
+// Persistent (or one item per CTA) two-tile kernel.  The producer takes work
+// items (from the ordered list when p.sched is set, else the CTA's own item)
+// and passes them to the other roles through a two-deep queue in shared
+// memory; it runs ahead into the next item's query and K/V tiles while the
+// current one finishes.  Barrier phases follow per-CTA counters of items (k)
+// and of K/V tiles (g), so they carry over from one item to the next.
 template <int D>
 __global__ void __launch_bounds__(kPpThreads, 1)
     paged_prefill_pp_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
@@ -473,40 +643,37 @@ __global__ void __launch_bounds__(kPpThreads, 1)
                             const __grid_constant__ CUtensorMap tmV) {
   using S = PpSmem<D>;
   constexpr int R = S::kRing;
+  constexpr int kBoxes = kPpKv / kStageTokens;  // 16-token boxes per K/V tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = bars + 1 + R;
-  uint64_t* s_full = bars + 1 + 2 * R;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = bars + 2 + R;
+  uint64_t* s_full = bars + 2 + 2 * R;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = s_full + 4;
-  uint64_t* done = s_full + 6;
+  uint64_t* item_full = s_full + 6;
+  uint64_t* item_empty = s_full + 8;
+  uint64_t* done = s_full + 10;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
+  __shared__ int s_item[2];
 
   if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
-  const int kvh = blockIdx.x;
-  const int qt = gridDim.y - 1 - blockIdx.y;  // the longest tiles of a sequence first
-  const int b = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G, TQ = p.TQ;
-  const int q0 = p.cu_q[b];
-  const int Q = p.cu_q[b + 1] - q0;
-  const int i0 = qt * 2 * TQ;
-  if (i0 >= Q) return;
-  int L = p.seq_lens[b];
-  const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
-  if (L > Lcap || Q > L) {
-    if (threadIdx.x == 0 && qt == 0 && kvh == 0) flag_error(PKV_DEVERR_SEQLEN);
-    if (Q > min(L, Lcap)) return;  // no consistent reading: rows are left unwritten
-    L = Lcap;
+  const bool persistent = p.sched != nullptr;
+  int own_item = -1;
+  if (!persistent) {
+    // One item per CTA: the longest query tiles of a sequence first.
+    own_item = ((int)blockIdx.z * p.nqt + (p.nqt - 1 - (int)blockIdx.y)) * p.Hkv + (int)blockIdx.x;
+    const PpItem it = pp_item(p, own_item);
+    if (threadIdx.x == 0 && it.bad_len && it.i0 == 0 && it.kvh == 0) flag_error(PKV_DEVERR_SEQLEN);
+    if (it.n_kv == 0) return;
   }
-  const int ctx = L - Q;
-  const int kv_end = ctx + min(Q, i0 + 2 * TQ);  // tokens any row of the CTA sees
-  const int n_kv = (kv_end + kPpKv - 1) / kPpKv;
 
   if (warp == 9) {
     tmem_alloc(&s_tmem, S::kCols);
@@ -515,14 +682,17 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   if (threadIdx.x == 0) {
     s_abort = 0;
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < R; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 4);  // one arrival per softmax warp
       mbar_init(&o_full[t], 1);
+      mbar_init(&item_full[t], 1);
+      mbar_init(&item_empty[t], 9);  // 8 softmax warps + the MMA warp
     }
     mbar_init(done, 1);
     fence_mbar_init();
@@ -533,33 +703,48 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   const uint32_t tmem = s_tmem;
   uint8_t* q_smem = smem + S::kOffQ;
   uint8_t* ring = smem + S::kOffRing;
+  if (warp < 8) regs_inc<kPpRegsSoftmax>();
+  else regs_dec<kPpRegsIo>();
+
+  // Consumers: the next item from the queue (-1: no more), released at once.
+  auto pop_item = [&](int k, int& item) -> bool {
+    if (!pp_wait_warp(&item_full[k & 1], (uint32_t)((k >> 1) & 1), &s_abort)) return false;
+    item = *reinterpret_cast<volatile int*>(&s_item[k & 1]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[k & 1]);
+    return true;
+  };
 
   if (warp < 8) {
     // ---- softmax of tile t = warp / 4; thread = row r ----
     const int t = warp / 4;
     const int r = threadIdx.x % 128;
-    const int i = i0 + t * TQ + r / G, g = r % G;
-    const bool row_valid = i < Q;
-    const int visible = min(ctx + i + 1, kv_end);
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
-    const uint32_t s_tm = tmem + 128u * t + lane_base;
+    const uint32_t s_tm = tmem + S::kSCol + 128u * t + lane_base;
     const uint32_t o_tm = tmem + S::kOCol + (uint32_t)D * t + lane_base;
     const float cl2 = p.scale_log2;
     const bool pos = cl2 >= 0.f;
-    float m_run = -INFINITY, l_run = 0.f;
+    int g = 0;  // K/V tiles before this item
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!(ok = pp_wait_warp(&s_full[t], (uint32_t)(j & 1), &s_abort))) break;
-      tc_fence_after_sync();
-      pp_softmax_tile<D>(s_tm, o_tm, j, visible, cl2, pos, m_run, l_run);
-      tc_fence_before_sync();
-      mbar_arrive(&p_full[t]);
-    }
-    if (ok) ok = pp_wait_warp(&o_full[t], (uint32_t)((n_kv - 1) & 1), &s_abort);
-    if (ok) {
+    for (int k = 0; ok; ++k) {
+      int item;
+      if (!(ok = pop_item(k, item)) || item < 0) break;
+      const PpItem it = pp_item(p, item);
+      const int i = it.i0 + t * TQ + r / G, gh = r % G;
+      const bool row_valid = i < it.Q;
+      const int visible = min(it.ctx + i + 1, it.kv_end);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < it.n_kv; ++j) {
+        if (!(ok = pp_wait_warp(&s_full[t], (uint32_t)((g + j) & 1), &s_abort))) break;
+        tc_fence_after_sync();
+        pp_softmax_tile<D>(s_tm, o_tm, j, visible, cl2, pos, m_run, l_run);
+        pp_warp_arrive(&p_full[t]);
+      }
+      if (ok) ok = pp_wait_warp(&o_full[t], (uint32_t)((g + it.n_kv - 1) & 1), &s_abort);
+      if (!ok) break;
       tc_fence_after_sync();
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.out) +
-                            ((size_t)(q0 + i) * p.Hq + (size_t)kvh * G + g) * D;
+                            ((size_t)(it.q0 + i) * p.Hq + (size_t)it.kvh * G + gh) * D;
       const float inv = 1.f / l_run;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -578,134 +763,174 @@ __global__ void __launch_bounds__(kPpThreads, 1)
           }
         }
       }
+      g += it.n_kv;
     }
   } else if (warp == 8) {
     // ---- producer ----
     const uint64_t pol = l2_policy_evict_first();
-    const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks;
     if (lane == 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * S::kQTile);
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int sb = 0; sb < S::SUB; ++sb)
-          tma_load_3d(q_smem + t * S::kQTile + sb * (kPrefillRows * 128), &tmQ, q_full, sb * 64,
-                      kvh * G, q0 + i0 + t * TQ, pol);
     }
-    int issued = 0;
-    int row = p.num_blocks * p.bs;  // box row of this lane's 16 tokens (past the end: zeros)
-    for (int idx = 0; idx < 2 * n_kv; ++idx) {
-      const int j = idx >> 1, slot = idx % R;
-      if ((idx & 1) == 0 && lane < kPpKv / kStageTokens) {
-        const int t0 = j * kPpKv + lane * kStageTokens;
-        row = p.num_blocks * p.bs;
-        if (t0 < kv_end) {
-          const int id = bt_row[t0 / p.bs];
-          if (id >= 0 && id < p.num_blocks) row = id * p.bs + t0 % p.bs;
-          else flag_error(PKV_DEVERR_BLOCK_ID);
+    int kv_idx = 0;  // K/V ring loads issued so far (K and V of each tile)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int item = -1;
+      if (persistent) {
+        if (lane == 0) {
+          const int n = atomicAdd(p.sched, 1);
+          item = n < p.sched[1] ? p.sched[2 + n] : -1;
+        }
+        item = __shfl_sync(kFull, item, 0);
+      } else {
+        item = k == 0 ? own_item : -1;
+      }
+      if (!(ok = pp_wait_warp(&item_empty[k & 1], (uint32_t)(((k >> 1) & 1) ^ 1), &s_abort))) break;
+      if (lane == 0) {
+        s_item[k & 1] = item;
+        mbar_arrive(&item_full[k & 1]);  // release: the store above is seen with the phase
+      }
+      if (item < 0) break;
+      const PpItem it = pp_item(p, item);
+      // The query tiles, once the previous item's last S MMA has read the old ones.
+      if (k > 0 && !(ok = pp_wait_warp(q_empty, (uint32_t)((k - 1) & 1), &s_abort))) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, 2 * S::kQTile);
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int sb = 0; sb < S::SUB; ++sb)
+            tma_load_3d(q_smem + t * S::kQTile + sb * (kPrefillRows * 128), &tmQ, q_full,
+                        sb * 64, it.kvh * G, it.q0 + it.i0 + t * TQ, pol);
+      }
+      const int32_t* bt_row = p.block_tables + (size_t)it.b * p.max_blocks;
+      int row = p.num_blocks * p.bs;  // box row of this lane's 16 tokens (past the end: zeros)
+      for (int e = 0; e < 2 * it.n_kv; ++e, ++kv_idx) {
+        const int j = e >> 1, slot = kv_idx % R;
+        if ((e & 1) == 0 && lane < kBoxes) {
+          const int t0 = j * kPpKv + lane * kStageTokens;
+          row = p.num_blocks * p.bs;
+          if (t0 < it.kv_end) {
+            const int id = bt_row[t0 / p.bs];
+            if (id >= 0 && id < p.num_blocks) row = id * p.bs + t0 % p.bs;
+            else flag_error(PKV_DEVERR_BLOCK_ID);
+          }
+        }
+        if (!(ok = pp_wait_warp(&kv_empty[slot], (uint32_t)(((kv_idx / R) & 1) ^ 1), &s_abort))) break;
+        if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], S::kKvTile);
+        __syncwarp();
+        if (lane < kBoxes) {
+          const CUtensorMap* map = (e & 1) ? &tmV : &tmK;
+#pragma unroll
+          for (int sb = 0; sb < S::SUB; ++sb)
+            tma_load_3d(ring + slot * S::kKvTile + sb * (kPpKv * 128) + lane * (kStageTokens * 128),
+                        map, &kv_full[slot], sb * 64, it.kvh, row, pol);
         }
       }
-      if (!pp_wait_warp(&kv_empty[slot], (uint32_t)(((idx / R) & 1) ^ 1), &s_abort)) break;
-      if (lane == 0) mbar_arrive_expect_tx(&kv_full[slot], S::kKvTile);
-      __syncwarp();
-      if (lane < kPpKv / kStageTokens) {
-        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
-#pragma unroll
-        for (int sb = 0; sb < S::SUB; ++sb)
-          tma_load_3d(ring + slot * S::kKvTile + sb * (kPpKv * 128) + lane * (kStageTokens * 128),
-                      map, &kv_full[slot], sb * 64, kvh, row, pol);
-      }
-      issued = idx + 1;
     }
     // Loads still in flight after an abort land before the CTA lets go of its
     // shared memory (bounded).
     if (s_abort && lane == 0)
-      for (int idx = max(0, issued - R); idx < issued; ++idx)
+      for (int idx = max(0, kv_idx - R); idx < kv_idx; ++idx)
         mbar_wait_bounded(&kv_full[idx % R], (uint32_t)((idx / R) & 1));
-  } else {
+  } else if (warp == 9) {
     // ---- MMA issuer ----
     constexpr uint32_t kIdescS = umma_idesc_bf16(kPrefillRows, kPpKv, false);
     constexpr uint32_t kIdescO = umma_idesc_bf16(kPrefillRows, D, true);
     const bool leader = lane == 0;
     const uint32_t q_addr = smem_u32(q_smem);
     const uint32_t ring_addr = smem_u32(ring);
-    auto issue_s = [&](int t, int j) {
-      const uint32_t k_addr = ring_addr + (uint32_t)(((2 * j) % R) * S::kKvTile);
+    auto issue_s = [&](int t, int kslot) {
+      const uint32_t k_addr = ring_addr + (uint32_t)(kslot * S::kKvTile);
       const uint32_t qa = q_addr + (uint32_t)(t * S::kQTile);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t ad = umma_desc_sw128(qa + (kk / 4) * (kPrefillRows * 128) + (kk % 4) * 32, 16, 1024);
         const uint64_t bd = umma_desc_sw128(k_addr + (kk / 4) * (kPpKv * 128) + (kk % 4) * 32, 16, 1024);
-        umma_bf16(tmem + 128u * t, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+        umma_bf16(tmem + S::kSCol + 128u * t, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[t]);
     };
-    auto issue_pv = [&](int t, int j) {
-      const uint32_t v_addr = ring_addr + (uint32_t)(((2 * j + 1) % R) * S::kKvTile);
+    auto issue_pv = [&](int t, int vslot, bool first) {
+      const uint32_t v_addr = ring_addr + (uint32_t)(vslot * S::kKvTile);
 #pragma unroll
       for (int kk = 0; kk < kPpKv / 16; ++kk) {
         const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, kPpKv * 128, 1024);
-        umma_bf16_tmem_a(tmem + S::kOCol + (uint32_t)D * t, tmem + 128u * t + 8u * kk, bd, kIdescO,
-                         (j > 0 || kk > 0) ? 1u : 0u);
+        umma_bf16_tmem_a(tmem + S::kOCol + (uint32_t)D * t, tmem + S::kSCol + 128u * t + 8u * kk,
+                         bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
       }
       umma_commit(&o_full[t]);
     };
-    bool ok = pp_wait_warp(q_full, 0, &s_abort) && pp_wait_warp(&kv_full[0], 0, &s_abort);
-    if (ok) {
-      tc_fence_after_sync();
-      if (leader) {
-        issue_s(0, 0);
-        issue_s(1, 0);
-        umma_commit(&kv_empty[0]);
-      }
-      __syncwarp();
-    }
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int iv = 2 * j + 1, ik = 2 * j + 2;
-      if (!(ok = pp_wait_warp(&kv_full[iv % R], (uint32_t)((iv / R) & 1), &s_abort))) break;
-      if (j == n_kv - 1 && kv_end < n_kv * kPpKv) {
-        // Tokens past the end: their V rows may hold anything (even NaN), and
-        // 0 * NaN must not reach O.
-        uint8_t* v_smem = ring + (iv % R) * S::kKvTile;
-        const int first = kv_end - j * kPpKv;
-        const int nvec = (kPpKv - first) * 8;
-        for (int sb = 0; sb < S::SUB; ++sb)
-          for (int v = lane; v < nvec; v += 32)
-            reinterpret_cast<uint4*>(v_smem + sb * (kPpKv * 128) + first * 128)[v] =
-                make_uint4(0u, 0u, 0u, 0u);
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
-      if (!(ok = pp_wait_warp(&p_full[0], (uint32_t)(j & 1), &s_abort))) break;
-      tc_fence_after_sync();
-      if (leader) issue_pv(0, j);
-      __syncwarp();
-      if (j + 1 < n_kv) {
-        if (!(ok = pp_wait_warp(&kv_full[ik % R], (uint32_t)((ik / R) & 1), &s_abort))) break;
-        if (!(ok = pp_wait_warp(&o_full[0], (uint32_t)(j & 1), &s_abort))) break;
-        tc_fence_after_sync();
-        if (leader) issue_s(0, j + 1);
-        __syncwarp();
-      }
-      if (!(ok = pp_wait_warp(&p_full[1], (uint32_t)(j & 1), &s_abort))) break;
-      tc_fence_after_sync();
-      if (leader) {
-        issue_pv(1, j);
-        umma_commit(&kv_empty[iv % R]);
-      }
-      __syncwarp();
-      if (j + 1 < n_kv) {
-        if (!(ok = pp_wait_warp(&o_full[1], (uint32_t)(j & 1), &s_abort))) break;
+    int g = 0, kv_idx = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int item;
+      if (!(ok = pop_item(k, item)) || item < 0) break;
+      const PpItem it = pp_item(p, item);
+      const int n = it.n_kv;
+      // S(0) of both tiles, once the query tiles and K_0 are in and (from the
+      // second item on) the previous P V has read the S / P columns.
+      if (!(ok = pp_wait_warp(q_full, (uint32_t)(k & 1), &s_abort))) break;
+      if (!(ok = pp_wait_warp(&kv_full[kv_idx % R], (uint32_t)((kv_idx / R) & 1), &s_abort))) break;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (g > 0 && !(ok = pp_wait_warp(&o_full[t], (uint32_t)((g - 1) & 1), &s_abort))) break;
         tc_fence_after_sync();
         if (leader) {
-          issue_s(1, j + 1);
-          umma_commit(&kv_empty[ik % R]);
+          issue_s(t, kv_idx % R);
+          if (t == 1) {
+            umma_commit(&kv_empty[kv_idx % R]);
+            if (n == 1) umma_commit(q_empty);
+          }
         }
         __syncwarp();
       }
+      if (!ok) break;
+      for (int j = 0; ok && j < n; ++j) {
+        const int iv = kv_idx + 2 * j + 1, ik = kv_idx + 2 * j + 2;
+        if (!(ok = pp_wait_warp(&kv_full[iv % R], (uint32_t)((iv / R) & 1), &s_abort))) break;
+        if (j == n - 1 && it.kv_end < n * kPpKv) {
+          // Tokens past the end: their V rows may hold anything (even NaN), and
+          // 0 * NaN must not reach O.
+          uint8_t* v_smem = ring + (iv % R) * S::kKvTile;
+          const int first = it.kv_end - j * kPpKv;
+          const int nvec = (kPpKv - first) * 8;
+          for (int sb = 0; sb < S::SUB; ++sb)
+            for (int v = lane; v < nvec; v += 32)
+              reinterpret_cast<uint4*>(v_smem + sb * (kPpKv * 128) + first * 128)[v] =
+                  make_uint4(0u, 0u, 0u, 0u);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (j + 1 < n && !(ok = pp_wait_warp(&kv_full[ik % R], (uint32_t)((ik / R) & 1), &s_abort)))
+          break;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          // P_t V_j, then S_t(j+1) over the columns it read once it is done.
+          if (!(ok = pp_wait_warp(&p_full[t], (uint32_t)((g + j) & 1), &s_abort))) break;
+          tc_fence_after_sync();
+          if (leader) {
+            issue_pv(t, iv % R, j == 0);
+            if (t == 1) umma_commit(&kv_empty[iv % R]);
+          }
+          __syncwarp();
+          if (j + 1 < n) {
+            if (!(ok = pp_wait_warp(&o_full[t], (uint32_t)((g + j) & 1), &s_abort))) break;
+            tc_fence_after_sync();
+            if (leader) {
+              issue_s(t, ik % R);
+              if (t == 1) {
+                umma_commit(&kv_empty[ik % R]);
+                if (j + 2 == n) umma_commit(q_empty);  // the item's last S
+              }
+            }
+            __syncwarp();
+          }
+        }
+      }
+      g += n;
+      kv_idx += 2 * n;
     }
     // Every MMA issued has finished before TMEM is released (bounded).
     if (leader) {

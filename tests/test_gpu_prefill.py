@@ -35,20 +35,41 @@ def _run(Hq, Hkv, D, bs, lens, qlens, seed=3, scale=None):
                                 to_device(host["v_cache"], "bf16"),
                                 torch.from_numpy(wl.block_tables).cuda(),
                                 torch.from_numpy(seq).cuda(), torch.from_numpy(cu).cuda(),
-                                int(max(qlens)), int(seq.max()), scale)
+                                int(max(qlens)), int(seq.max()), scale,
+                                workspace=_workspace(len(lens), Hq, Hkv, int(max(qlens))))
     torch.cuda.synchronize()
     return widen(out), ref
 
 
-@pytest.fixture(autouse=True, params=["auto", "single_tile"])
+PATHS = ["persistent", "per_item", "single_tile"]
+_path = {"name": "persistent"}
+
+
+@pytest.fixture(autouse=True, params=PATHS)
 def path(request):
-    old = pkv.set_prefill_path(pkv.PKV_PREFILL_AUTO if request.param == "auto"
-                               else pkv.PKV_PREFILL_SINGLE_TILE)
+    old = pkv.set_prefill_path(pkv.PKV_PREFILL_SINGLE_TILE if request.param == "single_tile"
+                               else pkv.PKV_PREFILL_AUTO)
+    _path["name"] = request.param
     pkv.device_errors(clear=True)
     yield request.param
     torch.cuda.synchronize()
     pkv.set_prefill_path(old)
     assert pkv.device_errors() == 0
+
+
+_ws = {"buf": None}
+
+
+def _workspace(B, Hq, Hkv, max_q):
+    """Scratch for the persistent schedule: one buffer reused by every call (each call
+    rebuilds its schedule), filled with garbage when it is (re)allocated, since it needs no
+    initialisation; None on the per-item path."""
+    if _path["name"] == "per_item":
+        return None
+    n = pkv.paged_attention_prefill_workspace_size(B, Hq, Hkv, max_q) // 4 + 1
+    if _ws["buf"] is None or _ws["buf"].numel() < n:
+        _ws["buf"] = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    return _ws["buf"]
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4), (32, 4), (64, 8), (32, 2)])
@@ -83,7 +104,8 @@ def test_prefill_single_query_equals_decode():
     seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
     cu = torch.arange(4, dtype=torch.int32, device="cuda")
     out_p = torch.empty_like(q)
-    pkv.paged_attention_prefill(out_p, q, kc, vc, bt, seq, cu, 1, max(lens), wl.scale)
+    pkv.paged_attention_prefill(out_p, q, kc, vc, bt, seq, cu, 1, max(lens), wl.scale,
+                                workspace=_workspace(3, 32, 8, 1))
     ref = oracle.paged_decode(host["q"], host["k_cache"], host["v_cache"], wl.block_tables,
                               np.asarray(lens, np.int32), wl.scale)
     assert_attention_close(widen(out_p), ref, "bf16", "prefill Q=1")
@@ -118,3 +140,14 @@ def test_prefill_scales(scale):
     uniform weights over the visible prefix."""
     got, ref = _run(16, 4, 128, 16, [700, 130, 64], [200, 130, 5], seed=17, scale=scale)
     assert_attention_close(got, ref, "bf16", f"scale={scale}")
+
+
+def test_prefill_workspace_reuse_across_calls():
+    """The shared workspace across calls with different batches in a row, with more work
+    items than the persistent grid has CTAs (each CTA takes several items)."""
+    if _path["name"] != "persistent":
+        pytest.skip("persistent schedule only")
+    for seed, lens, qlens in [(21, [500, 90, 3000, 70], [500, 90, 200, 1]),
+                              (22, [1200] * 12, [300] * 12)]:
+        got, ref = _run(32, 8, 128, 16, lens, qlens, seed=seed)
+        assert_attention_close(got, ref, "bf16", f"seed {seed}")
