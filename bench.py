@@ -64,28 +64,33 @@ def load_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha() -> str:
-    """Hash of the device-code sources (the .cuh files holding the kernels)."""
+KERNEL_SOURCES = {"decode": ("pkv_ptx.cuh", "pkv_decode.cuh"),
+                  "prefill": ("pkv_ptx.cuh", "pkv_decode.cuh", "pkv_prefill.cuh")}
+
+
+def kernel_source_sha(kind: str = "decode") -> str:
+    """Hash of the device-code sources a kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_344_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith(".cuh"):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(config: str, partition: int):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken on the
-    current kernel sources with the same partition length (else None)."""
-    path = os.path.join(ROOT, "profiles", f"decode_{config}_ncu.md")
+def recorded_traffic(config: str, partition: int, kind: str = "decode"):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel sources (and, for decode, the same partition length); else None."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_{config}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     s = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     q = re.search(r"partition_tokens:\s*([0-9]+)", text)
-    if not m or not s or not q or s.group(1) != kernel_source_sha() or int(q.group(1)) != partition:
+    if not m or not s or s.group(1) != kernel_source_sha(kind):
+        return None
+    if kind == "decode" and (not q or int(q.group(1)) != partition):
         return None
     return float(m.group(1))
 
@@ -546,7 +551,9 @@ def run_prefill(args, rank, world, local_rank):
                                    "Hq=32, Hkv=8, D=128, bs=16", "flops_per_step": flops},
             "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
-                         "traffic": None, "peak_source": src,
+                         "traffic": (recorded_traffic("chunked_append", 0, "prefill")
+                                     if args.prefill_kernel == "two_tile" else None),
+                         "peak_source": src,
                          "kernel": ("paged_prefill_kernel" if args.prefill_kernel == "single_tile"
                                     else "paged_prefill_pp_kernel"),
                          "schedule": args.prefill_kernel},
