@@ -839,26 +839,29 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     constexpr uint32_t kIdescS = umma_idesc_bf16(kPrefillRows, kPpKv, false);
     constexpr uint32_t kIdescO = umma_idesc_bf16(kPrefillRows, D, true);
     const bool leader = lane == 0;
-    const uint32_t q_addr = smem_u32(q_smem);
-    const uint32_t ring_addr = smem_u32(ring);
+    // Descriptors of the smem bases; an operand at byte offset o is base + o / 16
+    // (all of shared memory is below 2^18 bytes, so the 14-bit address field
+    // never carries).
+    const uint64_t q_desc = umma_desc_sw128(smem_u32(q_smem), 16, 1024);
+    const uint64_t k_desc = umma_desc_sw128(smem_u32(ring), 16, 1024);
+    const uint64_t v_desc = umma_desc_sw128(smem_u32(ring), kPpKv * 128, 1024);
     auto issue_s = [&](int t, int kslot) {
-      const uint32_t k_addr = ring_addr + (uint32_t)(kslot * S::kKvTile);
-      const uint32_t qa = q_addr + (uint32_t)(t * S::kQTile);
+      const uint64_t qd = q_desc + (uint64_t)((t * S::kQTile) >> 4);
+      const uint64_t kd = k_desc + (uint64_t)((kslot * S::kKvTile) >> 4);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t ad = umma_desc_sw128(qa + (kk / 4) * (kPrefillRows * 128) + (kk % 4) * 32, 16, 1024);
-        const uint64_t bd = umma_desc_sw128(k_addr + (kk / 4) * (kPpKv * 128) + (kk % 4) * 32, 16, 1024);
+        const uint64_t ad = qd + (uint64_t)(((kk / 4) * (kPrefillRows * 128) + (kk % 4) * 32) >> 4);
+        const uint64_t bd = kd + (uint64_t)(((kk / 4) * (kPpKv * 128) + (kk % 4) * 32) >> 4);
         umma_bf16(tmem + S::kSCol + 128u * t, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
       }
       umma_commit(&s_full[t]);
     };
     auto issue_pv = [&](int t, int vslot, bool first) {
-      const uint32_t v_addr = ring_addr + (uint32_t)(vslot * S::kKvTile);
+      const uint64_t vd = v_desc + (uint64_t)((vslot * S::kKvTile) >> 4);
 #pragma unroll
       for (int kk = 0; kk < kPpKv / 16; ++kk) {
-        const uint64_t bd = umma_desc_sw128(v_addr + kk * 16 * 128, kPpKv * 128, 1024);
         umma_bf16_tmem_a(tmem + S::kOCol + (uint32_t)D * t, tmem + S::kSCol + 128u * t + 8u * kk,
-                         bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
+                         vd + (uint64_t)((kk * 16 * 128) >> 4), kIdescO, (!first || kk > 0) ? 1u : 0u);
       }
       umma_commit(&o_full[t]);
     };
