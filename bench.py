@@ -538,6 +538,34 @@ def run_prefill(args, rank, world, local_rank):
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev_name)
     flops = workloads.prefill_flops(wl, cu_q)
     tflops = world * flops / (ms * 1e-3) / 1e12
+
+    # End to end through the same call: q from pinned host memory to the device, the
+    # attention, and out back to pinned host memory, every step, on the launching stream.
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty_like(q_host).pin_memory()
+    e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        q.copy_(q_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e_steps):
+        q.copy_(q_host, non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps, world, dev_name)
+    qbytes = q.numel() * q.element_size()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, f_s, n_s, cores = prefill_oracle_sample(wl, cu_q, dev, q, args.cpu_budget_flops)
+        cpu = {"value": round(f_s / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores,
+               "kind": "oracle",
+               "sample": f"multi-query attention of sequences 0..{n_s - 1} of {wl.B} "
+                         f"({f_s / 1e9:.1f} GFLOP), fp64, {dt:.2f} s"}
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             peak, src = float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (burst)"
@@ -557,7 +585,49 @@ def run_prefill(args, rank, world, local_rank):
                          "kernel": ("paged_prefill_kernel" if args.prefill_kernel == "single_tile"
                                     else "paged_prefill_pp_kernel"),
                          "schedule": args.prefill_kernel},
-            "gpu_launches": args.steps, "clocks": clocks.summary()}
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(world * flops / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": qbytes, "d2h_bytes_per_step": qbytes,
+                    "ms_per_step": round(e_ms, 4)},
+            "gpu_launches": args.steps * (2 if ws is not None else 1),
+            "clocks": clocks.summary()}
+
+
+def prefill_oracle_sample(wl, cu_q, dev, q, budget_flops: float):
+    """The fp64 oracle's multi-query attention on sequences 0..n-1 (cumulative causal flops
+    up to ``budget_flops``), over a compact host pool of just their blocks; returns
+    (seconds, flops, n, threads)."""
+    import torch
+    import oracle
+    sel, acc = [], 0
+    for b in range(wl.B):
+        L, Q = int(wl.seq_lens_pre[b]), int(cu_q[b + 1] - cu_q[b])
+        acc += 4 * wl.D * wl.Hq * ((L - Q) * Q + Q * (Q + 1) // 2)
+        sel.append(b)
+        if acc >= budget_flops:
+            break
+    kc, vc, tables, off = [], [], [], 0
+    nmax = max(-(-int(wl.seq_lens_pre[b]) // wl.bs) for b in sel)
+    for b in sel:
+        n = -(-int(wl.seq_lens_pre[b]) // wl.bs)
+        ids = torch.from_numpy(wl.block_tables[b, :n].astype(np.int64)).to(dev["k_cache"].device)
+        kc.append(dev["k_cache"][ids].cpu())
+        vc.append(dev["v_cache"][ids].cpu())
+        row = np.full(nmax, -1, np.int32)
+        row[:n] = np.arange(off, off + n, dtype=np.int32)
+        tables.append(row)
+        off += n
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    kc, vc = bits(torch.cat(kc)), bits(torch.cat(vc))
+    qh = bits(q[int(cu_q[0]):int(cu_q[len(sel)])].cpu())
+    cu = np.ascontiguousarray(cu_q[:len(sel) + 1] - cu_q[0]).astype(np.int32)
+    seq = np.ascontiguousarray(wl.seq_lens_pre[:len(sel)]).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.paged_prefill(qh, kc, vc, np.stack(tables), seq, cu, wl.scale)
+    return time.perf_counter() - t0, acc, len(sel), oracle.num_threads()
 
 
 def run_reference(args, rank, world):
@@ -602,6 +672,8 @@ def main():
     ap.add_argument("--cpu-budget-rows", type=int, default=400_000_000,
                     help="query-row x token budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-flops", type=float, default=1.5e10,
+                    help="prefill mode: causal flops of the oracle's timed sample")
     ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
                     help="decode step (default) or multi-query chunked-append attention")
     ap.add_argument("--prefill-kernel", choices=["two_tile", "per_item", "single_tile"],
