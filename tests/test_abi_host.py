@@ -147,3 +147,51 @@ def test_decode_path_selector(lib):
     assert pkv.set_decode_path(old) == pkv.PKV_PATH_CUDA_CORES
     with pytest.raises(pkv.PagedKVError):
         pkv.set_decode_path(9)
+
+
+def _prefill(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, bt=FAKE, mb=8, sl=FAKE, cu=FAKE, T=64, mq=32, msl=128, B=2, Hq=32,
+             Hkv=8, D=128, bs=16, nb=64, scale=0.088, dt=0, ws=None, wsb=0)
+    a.update(kw)
+    return lib.paged_attention_prefill(a["out"], a["q"], FAKE, FAKE, a["bt"], a["mb"], a["sl"],
+                                       a["cu"], a["T"], a["mq"], a["msl"], a["B"], a["Hq"],
+                                       a["Hkv"], a["D"], a["bs"], a["nb"], a["scale"], a["dt"],
+                                       a["ws"], a["wsb"], None)
+
+
+def test_prefill_workspace_size(lib):
+    # two query tiles of 128 / G tokens per work item: G = 4 -> 64 tokens per item
+    assert lib.paged_attention_prefill_workspace_size(2, 32, 8, 100) == (2 + 2 * 2 * 8) * 4
+    assert lib.paged_attention_prefill_workspace_size(3, 8, 8, 512) == (2 + 3 * 2 * 8) * 4
+    assert lib.paged_attention_prefill_workspace_size(0, 32, 8, 100) == 0
+    assert lib.paged_attention_prefill_workspace_size(2, 30, 8, 100) == 0  # Hq % Hkv != 0
+    assert lib.paged_attention_prefill_workspace_size(2, 32, 8, 0) == 0
+
+
+@host_only
+def test_prefill_rejects_bad_arguments(lib):
+    assert _prefill(lib, out=None) == ERR_ARG
+    assert _prefill(lib, q=FAKE + 8) == ERR_ARG  # misaligned
+    assert _prefill(lib, sl=FAKE + 2) == ERR_ARG
+    assert _prefill(lib, Hq=30) == ERR_ARG  # Hq % Hkv != 0
+    assert _prefill(lib, scale=float("inf")) == ERR_ARG
+    assert _prefill(lib, dt=1) == ERR_UNSUP  # fp32 has no tensor-core path here
+    assert _prefill(lib, D=96) == ERR_UNSUP
+    assert _prefill(lib, Hq=256, Hkv=8) == ERR_UNSUP  # G = 32
+    assert _prefill(lib, bs=8) == ERR_UNSUP
+    assert _prefill(lib, mq=0) == ERR_RANGE
+    assert _prefill(lib, mq=200) == ERR_RANGE  # longer than max_seq_len
+    assert _prefill(lib, msl=8 * 16 + 1) == ERR_RANGE  # more than the table holds
+    n = lib.paged_attention_prefill_workspace_size(2, 32, 8, 32)
+    assert _prefill(lib, ws=FAKE + 2, wsb=n) == ERR_ARG  # misaligned workspace
+    assert _prefill(lib, ws=FAKE, wsb=n - 4) == ERR_ARG  # too small
+    # empty calls succeed without touching the device
+    assert _prefill(lib, B=0) == 0
+    assert _prefill(lib, T=0) == 0
+
+
+def test_prefill_path_selector(lib):
+    old = pkv.set_prefill_path(pkv.PKV_PREFILL_SINGLE_TILE)
+    assert pkv.set_prefill_path(old) == pkv.PKV_PREFILL_SINGLE_TILE
+    with pytest.raises(pkv.PagedKVError):
+        pkv.set_prefill_path(4)
