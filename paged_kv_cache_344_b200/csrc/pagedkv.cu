@@ -521,7 +521,11 @@ int shared_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const int mc = std::max(1, 16 / G);
   const int64_t chunks = ceil_div(max_group_size, mc);
   const int64_t prefix_items = (int64_t)n_groups * chunks * shape.max_pp * Hkv;
-  const int64_t items = prefix_items + (int64_t)n_groups * max_group_size * shape.max_op * Hkv;
+  // A group whose members fit one MMA chunk is one CTA per KV head (prefix and
+  // own tokens together, no partials) unless the caller fixed a partition length.
+  const bool grouped = partition_size == 0 && max_group_size <= mc;
+  const int64_t items = grouped ? (int64_t)n_groups * Hkv
+                                : prefix_items + (int64_t)n_groups * max_group_size * shape.max_op * Hkv;
   if (items > 0x7fffffffLL) return PKV_ERR_OUT_OF_RANGE;
 
   if (step.k_new && (!step.v_new || !aligned16(step.k_new) || !aligned16(step.v_new) ||
@@ -566,6 +570,7 @@ int shared_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   sp.max_group = max_group_size;
   sp.P = shape.P;
   sp.n_prefix_items = (int)prefix_items;
+  sp.grouped = grouped ? 1 : 0;
 
   CUtensorMap mk, mv;
   const int64_t rows = num_blocks * block_size;

@@ -381,9 +381,25 @@ struct MmaConsumer {
   }
 
   __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane) {
+    consume_impl<false>(st, n_valid, lane, 0, GP);
+  }
+
+  // The same, with only query rows [r0, r1) of the N dimension scoring this
+  // stage (the others see it as masked): a stage of one member's own tokens in a
+  // shared-prefix group.  A row may then have seen no token yet, so the
+  // rescale factors are guarded against -inf - -inf.
+  __device__ __forceinline__ void consume_rows(uint8_t* st, int n_valid, int lane, int r0, int r1) {
+    consume_impl<true>(st, n_valid, lane, r0, r1);
+  }
+
+  template <bool kRows>
+  __device__ __forceinline__ void consume_impl(uint8_t* st, int n_valid, int lane, int r0, int r1) {
     const uint32_t sk = smem_u32(st);
     const uint32_t sv = sk + kTileBytes;
     const int mi = lane / 8, rr = lane % 8;
+    // With a row range, 8-row tiles outside it are skipped altogether: their
+    // state is what a fully masked stage would leave.
+    auto live = [&](int nt) { return !kRows || (nt * 8 < r1 && nt * 8 + 8 > r0); };
 
     // Scores: S = K Q^T, one m16n8k16 per (k-step, head tile).
     float s[NT][4];
@@ -398,7 +414,8 @@ struct MmaConsumer {
       uint32_t a[4];
       ldmatrix_x4(sk + (ks / 4) * kSubBytes + swz(row, chunk), a[0], a[1], a[2], a[3]);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+      for (int nt = 0; nt < NT; ++nt)
+        if (live(nt)) mma_bf16_16816(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
     }
 
     // Invalid tail slots of the last stage hold anything (even NaN): their
@@ -419,11 +436,20 @@ struct MmaConsumer {
     uint32_t pb[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
+      if (!live(nt)) {
+        pb[nt][0] = pb[nt][1] = 0u;
+        continue;
+      }
       float x[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int t = t0 + (j >> 1) * 8;
-        x[j] = (t < n_valid) ? s[nt][j] * scale_log2 : -INFINITY;
+        bool ok = t < n_valid;
+        if (kRows) {
+          const int n = nt * 8 + 2 * (lane % 4) + (j & 1);
+          ok = ok && n >= r0 && n < r1;
+        }
+        x[j] = ok ? s[nt][j] * scale_log2 : -INFINITY;
       }
       float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
 #pragma unroll
@@ -432,13 +458,25 @@ struct MmaConsumer {
         mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
       }
       const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
-      const float al0 = exp2f(m[nt][0] - mn0), al1 = exp2f(m[nt][1] - mn1);
+      float al0 = exp2f(m[nt][0] - mn0), al1 = exp2f(m[nt][1] - mn1);
+      if (kRows) {  // a row with no token so far keeps m = -inf and l = o = 0
+        al0 = mn0 == -INFINITY ? 1.f : al0;
+        al1 = mn1 == -INFINITY ? 1.f : al1;
+      }
       m[nt][0] = mn0;
       m[nt][1] = mn1;
-      x[0] = exp2f(x[0] - mn0);
-      x[1] = exp2f(x[1] - mn1);
-      x[2] = exp2f(x[2] - mn0);
-      x[3] = exp2f(x[3] - mn1);
+      if (kRows) {
+        const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
+        x[0] = exp2f(x[0] - b0);
+        x[1] = exp2f(x[1] - b1);
+        x[2] = exp2f(x[2] - b0);
+        x[3] = exp2f(x[3] - b1);
+      } else {
+        x[0] = exp2f(x[0] - mn0);
+        x[1] = exp2f(x[1] - mn1);
+        x[2] = exp2f(x[2] - mn0);
+        x[3] = exp2f(x[3] - mn1);
+      }
       float sum0 = x[0] + x[2], sum1 = x[1] + x[3];
 #pragma unroll
       for (int off = 4; off < 32; off *= 2) {
@@ -468,7 +506,8 @@ struct MmaConsumer {
       ldmatrix_x4_trans(sv + (d0 / 64) * kSubBytes + swz(t, (d0 % 64) / 8), a[0], a[1], a[2],
                         a[3]);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
+      for (int nt = 0; nt < NT; ++nt)
+        if (live(nt)) mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
     }
   }
 

@@ -43,6 +43,7 @@ struct SharedParams {
   int max_group;  // largest group size (upper bound)
   int P;          // partition length (tokens, multiple of 16)
   int n_prefix_items;
+  int grouped;    // 1: one CTA per (group, KV head), see group_piece
 };
 
 __device__ __forceinline__ int shared_len(const DecodeParams& d, int b) {
@@ -332,6 +333,177 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
   }
 }
 
+// One CTA for a whole group and one KV head, when the group's members fit the
+// 16 query rows of one MMA (members <= 16 / G).  The CTA's stages are the
+// shared prefix's (scored for every member's rows) followed by each member's
+// own tokens (scored for that member's rows only; the other rows see them as
+// masked).  The warps take stages round-robin, so each warp's running softmax
+// state covers some prefix stages and some own stages; merging the warps gives
+// every row exactly its prefix plus its own tokens.  No partials leave the CTA.
+template <class C, int D>
+__device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kvh, uint8_t* smem,
+                                            const CUtensorMap& tmK, const CUtensorMap& tmV) {
+  using T = __nv_bfloat16;
+  constexpr int kRing = DecodeSmem<C>::kRingBytes;
+  constexpr int kMaxMembers = 16;
+  static_assert(C::GP == 16, "group pieces use the 16-row consumer");
+  static_assert(kRing >= (2 * C::GP + C::GP * D) * 4, "state does not fit in the ring");
+  __shared__ int s_len[kMaxMembers], s_cum[kMaxMembers + 1];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kRing);
+  const DecodeParams& p = s.d;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int G = p.G;
+  T* out = reinterpret_cast<T*>(p.out);
+  const int lo = group_off(s, g), hi = max(lo, group_off(s, g + 1));
+  int members = hi - lo;
+  if (members <= 0) return;
+  const int mc = min(s.mc, kMaxMembers);
+  if (members > mc) {  // more members than the caller's bound: the rest stay unwritten
+    if (threadIdx.x == 0) flag_error(PKV_DEVERR_PREFIX);
+    members = mc;
+  }
+  const int plen = group_prefix(s, g, lo, hi);  // whole stages
+  if (p.k_new != nullptr) {
+    // Fused step: every member's new token (after any copy-on-write of its block)
+    // before anything is read.
+    for (int i = 0; i < members; ++i) {
+      const int L = shared_len(p, lo + i);
+      if (L > 0) fused_append<T, D>(p, lo + i, kvh, L);
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    int cum = plen / kStageTokens;
+    s_cum[0] = cum;
+    for (int i = 0; i < members; ++i) {
+      const int L = shared_len(p, lo + i);
+      s_len[i] = L;
+      cum += L > plen ? (L - plen + kStageTokens - 1) / kStageTokens : 0;
+      s_cum[i + 1] = cum;
+    }
+  }
+  __syncthreads();
+  {  // every member must hold the same physical blocks for the prefix
+    const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
+    const int nj = plen > 0 ? (plen - 1) / p.bs + 1 : 0;
+    for (int x = threadIdx.x; x < nj * members; x += blockDim.x) {
+      const int j = x % nj, b = lo + x / nj;
+      if (p.block_tables[(size_t)b * p.max_blocks + j] != r0[j]) flag_error(PKV_DEVERR_PREFIX);
+    }
+  }
+  const int n_pre = s_cum[0], n_all = s_cum[members];
+  // Stage k of the CTA: table row, first token, valid tokens, rows that score it.
+  auto stage_of = [&](int k, int& b, int& t0, int& nv, int& r0, int& r1) {
+    if (k < n_pre) {
+      b = lo;
+      t0 = k * kStageTokens;
+      nv = kStageTokens;
+      r0 = 0;
+      r1 = members * G;
+      return;
+    }
+    int i = 0;
+    while (k >= s_cum[i + 1]) ++i;
+    b = lo + i;
+    t0 = plen + (k - s_cum[i]) * kStageTokens;
+    nv = min(kStageTokens, s_len[i] - t0);
+    r0 = i * G;
+    r1 = r0 + G;
+  };
+  // This warp takes the CTA's stages warp, warp + kWarps, ...
+  const int first = warp, stride = kWarps;
+  const int n_w = n_all > first ? (n_all - first + stride - 1) / stride : 0;
+  uint8_t* ring = smem + warp * kRing;
+  uint64_t* wbar = bars + warp * C::kStages;
+  if (lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+#pragma unroll
+    for (int st = 0; st < C::kStages; ++st) mbar_init(&wbar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t pol = l2_policy_evict_first();
+  auto stage_id = [&](int kk) -> int {  // block id of the warp's kk-th stage
+    int b, t0, nv, r0, r1;
+    stage_of(first + stride * kk, b, t0, nv, r0, r1);
+    return p.block_tables[(size_t)b * p.max_blocks + t0 / p.bs];
+  };
+  int win_base = 0;
+  int win0 = lane < n_w ? stage_id(lane) : -1;
+  int win1 = 32 + lane < n_w ? stage_id(32 + lane) : -1;
+  auto issue = [&](int kk) {
+    if (kk - win_base >= 32) {
+      win0 = win1;
+      win_base += 32;
+      win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane) : -1;
+    }
+    const int id = __shfl_sync(kFull, win0, kk - win_base);  // kk - win_base < 32 here
+    if (lane == 0) {
+      int b, t0, nv, r0, r1;
+      stage_of(first + stride * kk, b, t0, nv, r0, r1);
+      const int st = kk % C::kStages;
+      int row;
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PKV_DEVERR_BLOCK_ID);
+        row = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
+      } else {
+        row = id * p.bs + t0 % p.bs;
+      }
+      mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
+      C::load_stage(ring + st * C::kStageBytes, &tmK, &tmV, &wbar[st], kvh, row, pol);
+    }
+  };
+  const int n_pro = n_w < C::kStages ? n_w : C::kStages;
+  for (int kk = 0; kk < n_pro; ++kk) issue(kk);
+
+  C c;
+  c.init_gather(p, lo, members, kvh, lane);
+  for (int kk = 0; kk < n_w; ++kk) {
+    const int st = kk % C::kStages;
+    const bool ok = mbar_wait_bounded(&wbar[st], (uint32_t)((kk / C::kStages) & 1));
+    if (__any_sync(kFull, !ok)) {
+      if (lane == 0) flag_error(PKV_DEVERR_TIMEOUT);
+      for (int j = kk; j < n_w && j < kk + C::kStages; ++j)
+        mbar_wait_bounded(&wbar[j % C::kStages], (uint32_t)((j / C::kStages) & 1));
+      break;
+    }
+    int b, t0, nv, r0, r1;
+    stage_of(first + stride * kk, b, t0, nv, r0, r1);
+    if (r0 == 0 && r1 == members * G)  // a prefix stage: every member's rows
+      c.consume(ring + st * C::kStageBytes, nv, lane);
+    else
+      c.consume_rows(ring + st * C::kStageBytes, nv, lane, r0, r1);
+    __syncwarp();
+    if (kk + C::kStages < n_w) issue(kk + C::kStages);
+  }
+
+  // Merge the warps; each row n = member * G + head goes to its sequence.  A row
+  // with no token at all (an empty sequence) is written as zeros.
+  c.store_state(reinterpret_cast<float*>(ring), lane);
+  __syncthreads();
+  constexpr int GP = C::GP;
+  const int rows = members * G;
+  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
+    const int n = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, reinterpret_cast<const float*>(smem + w * kRing)[n]);
+    float num = 0.f, den = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float* stt = reinterpret_cast<const float*>(smem + w * kRing);
+        const float f = exp2f(stt[n] - M);
+        num = fmaf(f, stt[2 * GP + n * D + d], num);
+        den = fmaf(f, stt[GP + n], den);
+      }
+    }
+    out[((size_t)(lo + n / G) * p.Hq + (size_t)kvh * G + n % G) * D + d] =
+        __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+  }
+}
+
 template <class C2, class C1, int D>
 __global__ void __launch_bounds__(kWarps * 32)
     paged_decode_shared_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
@@ -347,6 +519,10 @@ __global__ void __launch_bounds__(kWarps * 32)
     bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
     for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
     if (!ok) flag_error(PKV_DEVERR_PREFIX);
+  }
+  if (s.grouped) {
+    group_piece<C2, D>(s, (int)blockIdx.x / s.d.Hkv, (int)blockIdx.x % s.d.Hkv, smem, tmK, tmV);
+    return;
   }
   const SharedItem it = decode_shared_item(s, blockIdx.x);
   if (!it.valid) return;

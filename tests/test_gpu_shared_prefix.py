@@ -145,3 +145,37 @@ def test_broken_sharing_contract_is_flagged():
         wl.max_seq_len, wl.scale, torch.tensor([0, 2], dtype=torch.int32, device="cuda"),
         torch.tensor([64], dtype=torch.int32, device="cuda"), 4, workspace=ws)
     assert pkv.device_errors() & pkv.DEVERR_PREFIX
+
+
+@pytest.mark.parametrize("Hq,Hkv,mc", [(8, 8, 16), (16, 4, 4), (64, 8, 2), (32, 2, 1)])
+def test_grouped_pieces(Hq, Hkv, mc):
+    """Groups whose members fit one 16-row MMA run one CTA per (group, KV head): the prefix
+    stages and every member's own stages in one list, own stages scored for their member's
+    rows only.  Group sizes up to the limit, prefixes from 0 tokens, tails from 0 tokens,
+    and empty members; the split pieces (an explicit partition length) must agree."""
+    rng = np.random.default_rng(Hq * 7 + Hkv)
+    sizes = [int(x) for x in rng.integers(1, mc + 1, size=7)] + [mc]
+    shared = [int(x) * 16 for x in rng.integers(0, 14, size=len(sizes))]
+    tails = [int(x) for x in rng.integers(0, 90, size=sum(sizes))]
+    wl = workloads.grouped("grp", "bf16", Hq, Hkv, 128, 16, sizes, shared, tails, seed=21)
+    host = workloads.host_tensors(wl)
+    dev = _step_inputs(wl, host)
+    _, _, ref = oracle_step(wl, host)
+    for P in (0, 32):
+        out, _ = _run_shared(wl, dev, P)
+        assert_attention_close(widen(out), ref, wl.dtype, f"G={Hq // Hkv} P={P}")
+    # empty members in the one-CTA-per-group path
+    seq = dev["seq_lens"].clone()
+    empty = [0, wl.B - 1]
+    seq[empty] = 0
+    out, _ = _run_shared(wl, dev, 0, seq_lens=seq)
+    lens = wl.seq_lens_post.copy()
+    lens[empty] = 0
+    kc, vc = host["k_cache"].copy(), host["v_cache"].copy()
+    oracle.copy_blocks(kc, vc, wl.cow_pairs)
+    oracle.kv_write(host["k_new"], host["v_new"], kc, vc, wl.slot_mapping)
+    ref2 = oracle.paged_decode(host["q"], kc, vc, wl.block_tables, lens, wl.scale)
+    got = widen(out)
+    assert_attention_close(got, ref2, wl.dtype, "empty members")
+    assert np.all(got[empty] == 0.0)
+    assert pkv.device_errors() == 0
