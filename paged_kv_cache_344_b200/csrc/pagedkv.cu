@@ -301,6 +301,27 @@ int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap&
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
+// One CTA per (group, KV head), 16-row consumer with a ring of GROUP_STAGES
+// stages per warp (measured on B200, share workloads: 3 stages equal, 4 stages
+// (one CTA per SM) 1.6x slower).
+#ifndef PKV_GROUP_STAGES_D128
+#define PKV_GROUP_STAGES_D128 2
+#endif
+template <int D>
+int launch_group(const pkv::SharedParams& sp, int64_t items, const CUtensorMap& mk,
+                 const CUtensorMap& mv, cudaStream_t stream) {
+  constexpr int kStages = D == 128 ? PKV_GROUP_STAGES_D128 : pkv::MmaConsumer<D, 2>::kStages;
+  using C = pkv::MmaConsumer<D, 2, kStages>;
+  auto kernel = pkv::paged_decode_group_kernel<C, D>;
+  const size_t smem = pkv::DecodeSmem<C>::kBytes;
+  static std::atomic<uint64_t> smem_set{0};
+  int rc = ensure_smem(kernel, smem, smem_set);
+  if (rc != PKV_OK) return rc;
+  kernel<<<(unsigned)items, pkv::kWarps * 32, smem, stream>>>(sp, mk, mv);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PKV_OK : cuda_fail(e);
+}
+
 }  // namespace
 
 extern "C" {
@@ -570,12 +591,16 @@ int shared_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   sp.max_group = max_group_size;
   sp.P = shape.P;
   sp.n_prefix_items = (int)prefix_items;
-  sp.grouped = grouped ? 1 : 0;
 
   CUtensorMap mk, mv;
   const int64_t rows = num_blocks * block_size;
   if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
   if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
+  if (grouped) {
+    if (D == 64) return launch_group<64>(sp, items, mk, mv, stream);
+    if (D == 128) return launch_group<128>(sp, items, mk, mv, stream);
+    return launch_group<256>(sp, items, mk, mv, stream);
+  }
   if (G <= 8) {
     if (D == 64) return launch_shared<64, 1>(sp, items, mk, mv, stream);
     if (D == 128) return launch_shared<128, 1>(sp, items, mk, mv, stream);

@@ -291,13 +291,13 @@ struct SimtConsumer {
 #define PKV_MMA_STAGES_D128 2
 #endif
 
-template <int D, int NT>
+template <int D, int NT, int STAGES = (D <= 64 ? 6 : (D <= 128 ? PKV_MMA_STAGES_D128 : 2))>
 struct MmaConsumer {
   static constexpr int SUB = D / 64;
   static constexpr int kSubBytes = kStageTokens * 128;
   static constexpr int kTileBytes = SUB * kSubBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = D <= 64 ? 6 : (D <= 128 ? PKV_MMA_STAGES_D128 : 2);
+  static constexpr int kStages = STAGES;
   static constexpr int KS = D / 16;
   static constexpr int MT = D / 16;
   static constexpr int GP = 8 * NT;

@@ -43,7 +43,6 @@ struct SharedParams {
   int max_group;  // largest group size (upper bound)
   int P;          // partition length (tokens, multiple of 16)
   int n_prefix_items;
-  int grouped;    // 1: one CTA per (group, KV head), see group_piece
 };
 
 __device__ __forceinline__ int shared_len(const DecodeParams& d, int b) {
@@ -504,6 +503,23 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   }
 }
 
+// One CTA per (group, KV head): group_piece with consumer C (16 rows).
+template <class C, int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    paged_decode_group_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
+                              const __grid_constant__ CUtensorMap tmV) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {  // the groups must tile the batch in order
+    bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
+    for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
+    if (!ok) flag_error(PKV_DEVERR_PREFIX);
+  }
+  group_piece<C, D>(s, (int)blockIdx.x / s.d.Hkv, (int)blockIdx.x % s.d.Hkv, smem, tmK, tmV);
+}
+
 template <class C2, class C1, int D>
 __global__ void __launch_bounds__(kWarps * 32)
     paged_decode_shared_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
@@ -519,10 +535,6 @@ __global__ void __launch_bounds__(kWarps * 32)
     bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
     for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
     if (!ok) flag_error(PKV_DEVERR_PREFIX);
-  }
-  if (s.grouped) {
-    group_piece<C2, D>(s, (int)blockIdx.x / s.d.Hkv, (int)blockIdx.x % s.d.Hkv, smem, tmK, tmV);
-    return;
   }
   const SharedItem it = decode_shared_item(s, blockIdx.x);
   if (!it.valid) return;
