@@ -235,7 +235,10 @@ int paged_decode_step(void *out, const void *q, const void *k_new, const void *v
  * member.  Prefix pieces score one read of the shared K/V against the queries
  * of up to 16 / G members at once, stacked in the tensor-core N dimension.
  * Pieces over each sequence's own tokens follow, as in paged_attention_decode.
- * The pieces' partials are merged in the same launch.
+ * The pieces' partials are merged in the same launch.  When partition_size is
+ * 0 and max_group_size <= 16 / G, each (group, KV head) is instead one CTA that
+ * reads the prefix once and every member's own tokens, with no partials (the
+ * workspace is then left untouched, but must still be passed).
  *   group_offsets  device [n_groups + 1] int32: group g is sequences
  *                  group_offsets[g] .. group_offsets[g+1]-1.  The offsets start
  *                  at 0, end at B and never decrease (a group may have one member).
