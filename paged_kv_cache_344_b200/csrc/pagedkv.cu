@@ -301,23 +301,28 @@ int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap&
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
-// One CTA per (group, KV head), 16-row consumer with a ring of GROUP_STAGES
-// stages per warp (measured on B200, share workloads: 3 stages equal, 4 stages
-// (one CTA per SM) 1.6x slower).
+// One CTA of GROUP_WARPS warps per (group, KV head), 16-row consumer with a
+// ring of GROUP_STAGES stages per warp.  Measured on B200 (share workloads):
+// 6 warps (2 CTAs per SM) beat 4 by up to 7% and 8 (1 CTA per SM) are 1.3x
+// slower; 3 stages equal 2, 4 stages (1 CTA per SM) are 1.6x slower.
 #ifndef PKV_GROUP_STAGES_D128
 #define PKV_GROUP_STAGES_D128 2
+#endif
+#ifndef PKV_GROUP_WARPS
+#define PKV_GROUP_WARPS 6
 #endif
 template <int D>
 int launch_group(const pkv::SharedParams& sp, int64_t items, const CUtensorMap& mk,
                  const CUtensorMap& mv, cudaStream_t stream) {
   constexpr int kStages = D == 128 ? PKV_GROUP_STAGES_D128 : pkv::MmaConsumer<D, 2>::kStages;
+  constexpr int W = PKV_GROUP_WARPS;
   using C = pkv::MmaConsumer<D, 2, kStages>;
-  auto kernel = pkv::paged_decode_group_kernel<C, D>;
-  const size_t smem = pkv::DecodeSmem<C>::kBytes;
+  auto kernel = pkv::paged_decode_group_kernel<C, D, W>;
+  const size_t smem = pkv::GroupSmem<C, D, W>::kBytes;
   static std::atomic<uint64_t> smem_set{0};
   int rc = ensure_smem(kernel, smem, smem_set);
   if (rc != PKV_OK) return rc;
-  kernel<<<(unsigned)items, pkv::kWarps * 32, smem, stream>>>(sp, mk, mv);
+  kernel<<<(unsigned)items, W * 32, smem, stream>>>(sp, mk, mv);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }

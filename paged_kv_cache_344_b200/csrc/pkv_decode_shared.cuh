@@ -339,7 +339,7 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
 // masked).  The warps take stages round-robin, so each warp's running softmax
 // state covers some prefix stages and some own stages; merging the warps gives
 // every row exactly its prefix plus its own tokens.  No partials leave the CTA.
-template <class C, int D>
+template <class C, int D, int W>
 __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kvh, uint8_t* smem,
                                             const CUtensorMap& tmK, const CUtensorMap& tmV) {
   using T = __nv_bfloat16;
@@ -348,7 +348,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   static_assert(C::GP == 16, "group pieces use the 16-row consumer");
   static_assert(kRing >= (2 * C::GP + C::GP * D) * 4, "state does not fit in the ring");
   __shared__ int s_len[kMaxMembers], s_cum[kMaxMembers + 1];
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kWarps * kRing);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * kRing);
   const DecodeParams& p = s.d;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
@@ -409,8 +409,8 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     r0 = i * G;
     r1 = r0 + G;
   };
-  // This warp takes the CTA's stages warp, warp + kWarps, ...
-  const int first = warp, stride = kWarps;
+  // This warp takes the CTA's stages warp, warp + W, ...
+  const int first = warp, stride = W;
   const int n_w = n_all > first ? (n_all - first + stride - 1) / stride : 0;
   uint8_t* ring = smem + warp * kRing;
   uint64_t* wbar = bars + warp * C::kStages;
@@ -487,11 +487,11 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     const int n = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, reinterpret_cast<const float*>(smem + w * kRing)[n]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, reinterpret_cast<const float*>(smem + w * kRing)[n]);
     float num = 0.f, den = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
+      for (int w = 0; w < W; ++w) {
         const float* stt = reinterpret_cast<const float*>(smem + w * kRing);
         const float f = exp2f(stt[n] - M);
         num = fmaf(f, stt[2 * GP + n * D + d], num);
@@ -503,9 +503,15 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   }
 }
 
-// One CTA per (group, KV head): group_piece with consumer C (16 rows).
-template <class C, int D>
-__global__ void __launch_bounds__(kWarps * 32)
+// One CTA of W warps per (group, KV head): group_piece with consumer C (16 rows).
+template <class C, int D, int W>
+struct GroupSmem {
+  static constexpr size_t kBytes =
+      1024 /*alignment slack*/ + (size_t)W * DecodeSmem<C>::kRingBytes + W * C::kStages * 8;
+};
+
+template <class C, int D, int W>
+__global__ void __launch_bounds__(W * 32)
     paged_decode_group_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
                               const __grid_constant__ CUtensorMap tmV) {
   extern __shared__ uint8_t smem_raw[];
@@ -517,7 +523,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
     if (!ok) flag_error(PKV_DEVERR_PREFIX);
   }
-  group_piece<C, D>(s, (int)blockIdx.x / s.d.Hkv, (int)blockIdx.x % s.d.Hkv, smem, tmK, tmV);
+  group_piece<C, D, W>(s, (int)blockIdx.x / s.d.Hkv, (int)blockIdx.x % s.d.Hkv, smem, tmK, tmV);
 }
 
 template <class C2, class C1, int D>
