@@ -151,3 +151,47 @@ def test_prefill_workspace_reuse_across_calls():
                               (22, [1200] * 12, [300] * 12)]:
         got, ref = _run(32, 8, 128, 16, lens, qlens, seed=seed)
         assert_attention_close(got, ref, "bf16", f"seed {seed}")
+
+
+def test_prefill_device_checks_flag_and_stay_in_bounds():
+    """Out-of-range block ids are flagged and read as zeros (the rest of the batch is exact);
+    a sequence with more queries than tokens is flagged and its rows are left as they were."""
+    lens, qlens = [200, 90, 50], [40, 30, 60]  # sequence 2 has Q > L
+    wl = workloads.custom("pf", "bf16", 3, 32, 8, 128, 16, lens, seed=31)
+    host = workloads.host_tensors(wl)
+    rng = np.random.default_rng(32)
+    cu = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = torch.from_numpy(rng.standard_normal((int(cu[-1]), 32, 128), dtype=np.float32))
+    q = q.to(torch.bfloat16)
+    bt = wl.block_tables.copy()
+    bt[0, 3] = wl.num_blocks + 7  # sequence 0: one block id out of range
+    seq = np.asarray(lens, np.int32)
+    out = torch.full_like(q, 3.0).cuda()
+    pkv.device_errors(clear=True)
+    pkv.paged_attention_prefill(out, q.cuda(), to_device(host["k_cache"], "bf16"),
+                                to_device(host["v_cache"], "bf16"), torch.from_numpy(bt).cuda(),
+                                torch.from_numpy(seq).cuda(), torch.from_numpy(cu).cuda(),
+                                max(qlens), max(lens), wl.scale,
+                                workspace=_workspace(3, 32, 8, max(qlens)))
+    torch.cuda.synchronize()
+    bits = pkv.device_errors(clear=True)
+    assert bits & pkv.DEVERR_BLOCK_ID and bits & pkv.DEVERR_SEQLEN
+    got = widen(out)
+    assert np.isfinite(got).all()
+    # sequence 2's rows are untouched
+    assert np.all(got[cu[2]:cu[3]] == 3.0)
+    # sequence 1 (valid table, valid lengths) is exact
+    q_bits = q.view(torch.int16).numpy().view(np.uint16)
+    ref = oracle.paged_prefill(np.ascontiguousarray(q_bits[cu[1]:cu[2]]), host["k_cache"],
+                               host["v_cache"], np.ascontiguousarray(wl.block_tables[1:2]),
+                               seq[1:2], np.array([0, qlens[1]], np.int32), wl.scale)
+    assert_attention_close(got[cu[1]:cu[2]], ref, "bf16", "valid sequence beside bad ones")
+    # sequence 0 equals attention with that block read as zeros
+    kz, vz = host["k_cache"].copy(), host["v_cache"].copy()
+    bad = wl.block_tables[0, 3]
+    kz[bad] = 0
+    vz[bad] = 0
+    ref0 = oracle.paged_prefill(np.ascontiguousarray(q_bits[cu[0]:cu[1]]), kz, vz,
+                                np.ascontiguousarray(wl.block_tables[0:1]), seq[0:1],
+                                np.array([0, qlens[0]], np.int32), wl.scale)
+    assert_attention_close(got[cu[0]:cu[1]], ref0, "bf16", "bad block read as zeros")
