@@ -425,32 +425,6 @@ __device__ __forceinline__ void pp_warp_arrive(uint64_t* bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
-// 2^x for a pair, on the FMA pipe instead of the special-function unit:
-// x = n + f with n = round(x) (the 1.5 * 2^23 addition leaves n in the low
-// mantissa bits of t) and f in [-1/2, 1/2]; 2^f is a cubic, fitted here
-// (minimax over [-1/2, 1/2], relative error 7.5e-5, below bf16's 2^-9); 2^n is
-// added to its exponent field.  x is clamped at -126 (2^-126 is zero at the
-// precision P keeps); NaN stays NaN.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  x.x = x.x < -126.f ? -126.f : x.x;
-  x.y = x.y < -126.f ? -126.f : x.y;
-  const float2 t = fadd2(x, make_float2(kRound, kRound));
-  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-  float2 q = ffma2(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.242611125f, 0.242611125f));
-  q = ffma2(q, f, make_float2(0.693260968f, 0.693260968f));
-  q = ffma2(q, f, make_float2(0.999928057f, 0.999928057f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
-
-// Of every 8 pairs of probabilities, kPpPolyPairs take exp2_poly2 (the rest
-// the special-function unit).
-#ifndef PKV_PP_POLY_PAIRS
-#define PKV_PP_POLY_PAIRS 0
-#endif
-constexpr int kPpPolyPairs = PKV_PP_POLY_PAIRS;
 
 // One K/V tile of the row softmax for the thread's row: read S_t(j), compute P
 // and the running max / sum, rescale O if the max moved (the issuer computed
@@ -513,12 +487,8 @@ __device__ __forceinline__ void pp_softmax_tile(uint32_t s_tm, uint32_t o_tm, in
   for (int c = 0; c < kPpKv; c += 2) {
     const float2 e = ffma2(make_float2(x[c], x[c + 1]), kk2, nm2);
     float2 pr;
-    if ((c / 2) % 8 < kPpPolyPairs) {
-      pr = exp2_poly2(e);
-    } else {
-      pr.x = ex2_approx(e.x);
-      pr.y = ex2_approx(e.y);
-    }
+    pr.x = ex2_approx(e.x);
+    pr.y = ex2_approx(e.y);
     acc[(c / 2) % (kAcc / 2)] = fadd2(acc[(c / 2) % (kAcc / 2)], pr);
     pk[c / 64][(c % 64) / 2] = pack_bf16x2(pr.x, pr.y);
   }
