@@ -354,6 +354,19 @@ int pkv_last_cuda_error(void);
 int pkv_device_errors(uint32_t *bits, int clear);
 
 /*
+ * Self-test of the pipelines' time limit.  Launches (on `stream`) one kernel
+ * whose single thread waits, with the bounded wait that every TMA / MMA
+ * pipeline of this library uses, on a barrier that nothing completes.  After
+ * 2^30 SM cycles (about 0.55 s at 1.965 GHz) the wait gives up and sets
+ * PKV_DEVERR_TIMEOUT; the device stays usable.  While that bit is set, every
+ * CTA of every attention launch (decode, shared-prefix decode, prefill) returns
+ * at once, whole, without reading or writing anything, so that one stall does
+ * not become a wait per CTA; pkv_device_errors(&bits, 1) clears it.  Returns
+ * PKV_OK or PKV_ERR_CUDA (launch failure).
+ */
+int pkv_debug_stalled_wait(pkv_stream_t stream);
+
+/*
  * Arithmetic units used by paged_attention_decode, set for the whole process
  * (for testing and measuring both kernels):
  *   PKV_PATH_AUTO          every bf16 call on tensor cores, fp32 on CUDA cores;

@@ -112,6 +112,8 @@ def lib() -> ctypes.CDLL:
     L.pkv_set_prefill_path.restype = i32
     L.pkv_set_decode_path.argtypes = [i32]
     L.pkv_set_decode_path.restype = i32
+    L.pkv_debug_stalled_wait.argtypes = [ctypes.c_void_p]
+    L.pkv_debug_stalled_wait.restype = i32
     L.pkv_set_decode_split.argtypes = [i32]
     L.pkv_set_decode_split.restype = i32
     L.pkv_set_decode_ctas.argtypes = [i32]
@@ -293,6 +295,16 @@ def device_errors(clear: bool = True) -> int:
     bits = ctypes.c_uint32(0)
     _check("pkv_device_errors", lib().pkv_device_errors(ctypes.byref(bits), int(clear)))
     return int(bits.value)
+
+
+def debug_stalled_wait(stream=None) -> None:
+    """Launch the time-limit self-test: one bounded wait that nothing satisfies gives up
+    after about half a second and sets DEVERR_TIMEOUT (which stops later attention
+    launches until device_errors(clear=True))."""
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    _check("pkv_debug_stalled_wait", lib().pkv_debug_stalled_wait(
+        ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))))
 
 
 def set_decode_path(mode: int) -> int:

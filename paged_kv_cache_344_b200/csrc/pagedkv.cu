@@ -888,6 +888,26 @@ int pkv_set_decode_ctas(int ctas) {
   return g_decode_ctas.exchange(ctas);
 }
 
+namespace pkv {
+// One thread waits, with the bounded wait of every pipeline, on a barrier that
+// nothing completes; it gives up after the time limit and flags the timeout.
+__global__ void stalled_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_bounded(&bar, 0)) flag_error(PKV_DEVERR_TIMEOUT);
+  }
+}
+}  // namespace pkv
+
+int pkv_debug_stalled_wait(pkv_stream_t stream_) {
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  pkv::stalled_wait_kernel<<<1, 32, 0, stream>>>();
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PKV_OK : cuda_fail(e);
+}
+
 int pkv_set_prefill_path(int mode) {
   if (mode != PKV_PREFILL_AUTO && mode != PKV_PREFILL_SINGLE_TILE) return PKV_ERR_INVALID_ARG;
   return g_prefill_path.exchange(mode);

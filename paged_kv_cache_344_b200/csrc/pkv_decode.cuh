@@ -39,6 +39,15 @@ __device__ uint32_t g_device_errors;  // OR of PKV_DEVERR_* bits
 
 __device__ __forceinline__ void flag_error(uint32_t bits) { atomicOr(&g_device_errors, bits); }
 
+// True once a pipeline wait has timed out anywhere on the device.  Thread 0 reads
+// the flag and one barrier hands its answer to the whole CTA, so a CTA stops whole
+// or runs whole: no barrier further on can miss a warp that returned early.
+__device__ __forceinline__ bool cta_timed_out() {
+  const bool t = threadIdx.x == 0 &&
+                 (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT);
+  return __syncthreads_or(t) != 0;
+}
+
 struct DecodeParams {
   void* out;
   const void* q;
@@ -652,7 +661,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int P = p.part_tokens;
 
   // After a pipeline timeout anywhere, later CTAs stop at once instead of waiting too.
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (cta_timed_out()) return;
   int L = p.seq_lens[b];
   const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
   if (L < 0 || L > Lcap) {

@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   int* s_pre = reinterpret_cast<int*>(bars + kWarps * NS);  // [B + 1]
   __shared__ int s_warp_tot[kWarps];
 
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (cta_timed_out()) return;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int B = p.B, Hkv = p.Hkv, G = p.G;

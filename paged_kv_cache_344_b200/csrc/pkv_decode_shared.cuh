@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(W * 32)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (cta_timed_out()) return;
   if (blockIdx.x == 0 && threadIdx.x == 0) {  // the groups must tile the batch in order
     bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
     for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ float s_M[16], s_den[16];
   __shared__ int s_last;
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (cta_timed_out()) return;
   if (blockIdx.x == 0 && threadIdx.x == 0) {  // the groups must tile the batch in order
     bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
     for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];

@@ -113,10 +113,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   uint64_t* bar_kv = bar_q + 1;  // [2]
   uint64_t* bar_s = bar_q + 3;
   uint64_t* bar_o = bar_q + 4;
+  uint64_t* bar_done = bar_q + 5;  // after a timeout: every MMA issued so far is complete
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (cta_timed_out()) return;
   const int kvh = blockIdx.x, qt = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     mbar_init(&bar_kv[1], 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
+    mbar_init(bar_done, 1);
     fence_mbar_init();
   }
   tc_fence_before_sync();
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   uint8_t* q_smem = smem + S::kOffQ;
   auto stage_ptr = [&](int st) { return smem + S::kOffStage + st * S::kStage; };
   const uint64_t pol = l2_policy_evict_first();
+  int n_issued = 0;  // K/V tiles whose loads thread 0 has issued
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmQ);
     prefetch_tensormap(&tmK);
@@ -178,6 +181,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     prefill_issue_kv<D>(p, stage_ptr(0), &tmK, &tmV, &bar_kv[0], bt_row, kvh, 0, kv_end, pol);
     if (n_kv > 1)
       prefill_issue_kv<D>(p, stage_ptr(1), &tmK, &tmV, &bar_kv[1], bt_row, kvh, 1, kv_end, pol);
+    n_issued = min(n_kv, 2);
   }
 
   constexpr uint32_t kIdescS = umma_idesc_bf16(kPrefillRows, kPrefillKv, false);
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       }
     }
     ok = mbar_wait_bounded(bar_s, (uint32_t)(j & 1));
-    if (__syncthreads_or(!ok)) break;
+    if (__syncthreads_or(!ok)) { ok = false; break; }  // the CTA agrees
     tc_fence_after_sync();
 
     // Row softmax over this tile (the warp reads its 32 lanes of S).
@@ -239,11 +243,13 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (j > 0) {
       // The previous P V must be done before O is rescaled and P / stage st^1 reused.
       ok = mbar_wait_bounded(bar_o, (uint32_t)((j - 1) & 1));
-      if (__syncthreads_or(!ok)) break;
+      if (__syncthreads_or(!ok)) { ok = false; break; }  // the CTA agrees
       tc_fence_after_sync();
-      if (threadIdx.x == 0 && j + 1 < n_kv)
+      if (threadIdx.x == 0 && j + 1 < n_kv) {
         prefill_issue_kv<D>(p, stage_ptr(st ^ 1), &tmK, &tmV, &bar_kv[st ^ 1], bt_row, kvh, j + 1,
                             kv_end, pol);
+        n_issued = j + 2;
+      }
       if (__any_sync(kFull, alpha != 1.f)) {
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -330,11 +336,15 @@ __global__ void __launch_bounds__(kWarps * 32)
     flag_error(PKV_DEVERR_TIMEOUT);
     s_abort = 1;
   }
-  // Free TMEM once every warp is done with it (and, after a timeout, once the
-  // MMAs issued so far have had their bounded chance to finish).
+  // Free TMEM and shared memory once every warp is done with them; after a
+  // timeout, once the MMAs and the loads issued so far have had their bounded
+  // chance to finish.
   if (!ok && threadIdx.x == 0) {
-    mbar_wait_bounded(bar_s, 0);
-    mbar_wait_bounded(bar_o, 0);
+    umma_commit(bar_done);
+    mbar_wait_bounded(bar_done, 0);
+    mbar_wait_bounded(bar_q, 0);
+    for (int jj = max(0, n_issued - 2); jj < n_issued; ++jj)
+      mbar_wait_bounded(&bar_kv[jj & 1], (uint32_t)((jj >> 1) & 1));
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -632,7 +642,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
   __shared__ volatile int s_abort;
   __shared__ int s_item[2];
 
-  if (*reinterpret_cast<volatile uint32_t*>(&g_device_errors) & PKV_DEVERR_TIMEOUT) return;
+  if (cta_timed_out()) return;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G, TQ = p.TQ;
   const bool persistent = p.sched != nullptr;
@@ -743,7 +753,8 @@ __global__ void __launch_bounds__(kPpThreads, 1)
       prefetch_tensormap(&tmK);
       prefetch_tensormap(&tmV);
     }
-    int kv_idx = 0;  // K/V ring loads issued so far (K and V of each tile)
+    int kv_idx = 0;   // K/V ring loads issued so far (K and V of each tile)
+    int q_loads = 0;  // query tile pairs issued so far
     bool ok = true;
     for (int k = 0; ok; ++k) {
       int item = -1;
@@ -774,6 +785,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
             tma_load_3d(q_smem + t * S::kQTile + sb * (kPrefillRows * 128), &tmQ, q_full,
                         sb * 64, it.kvh * G, it.q0 + it.i0 + t * TQ, pol);
       }
+      ++q_loads;
       const int32_t* bt_row = p.block_tables + (size_t)it.b * p.max_blocks;
       int row = p.num_blocks * p.bs;  // box row of this lane's 16 tokens (past the end: zeros)
       for (int e = 0; e < 2 * it.n_kv; ++e, ++kv_idx) {
@@ -801,9 +813,11 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     }
     // Loads still in flight after an abort land before the CTA lets go of its
     // shared memory (bounded).
-    if (s_abort && lane == 0)
+    if (s_abort && lane == 0) {
       for (int idx = max(0, kv_idx - R); idx < kv_idx; ++idx)
         mbar_wait_bounded(&kv_full[idx % R], (uint32_t)((idx / R) & 1));
+      if (q_loads > 0) mbar_wait_bounded(q_full, (uint32_t)((q_loads - 1) & 1));
+    }
   } else if (warp == 9) {
     // ---- MMA issuer ----
     constexpr uint32_t kIdescS = umma_idesc_bf16(kPrefillRows, kPpKv, false);
