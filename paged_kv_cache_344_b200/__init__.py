@@ -301,6 +301,7 @@ def debug_stalled_wait(stream=None) -> None:
     """Launch the time-limit self-test: one bounded wait that nothing satisfies gives up
     after about half a second and sets DEVERR_TIMEOUT (which stops later attention
     launches until device_errors(clear=True))."""
+    import torch
     if stream is None:
         stream = torch.cuda.current_stream()
     _check("pkv_debug_stalled_wait", lib().pkv_debug_stalled_wait(
