@@ -103,8 +103,10 @@ def test_stalled_wait_gives_up_and_attention_stands_down():
     for name, out, before, after in checks:
         assert bool((out == SENTINEL).all()), f"{name}: output written after a timeout"
         if before is not None:
-            assert torch.equal(before[0], after[0]) and torch.equal(before[1], after[1]), \
-                f"{name}: cache written after a timeout"
+            # bitwise (unused slots hold NaN)
+            same = all(torch.equal(x.view(torch.int16), y.view(torch.int16))
+                       for x, y in zip(before, after))
+            assert same, f"{name}: cache written after a timeout"
     # nothing else was flagged, and clearing works
     assert pkv.device_errors(clear=True) == pkv.DEVERR_TIMEOUT
     assert pkv.device_errors(clear=False) == 0
