@@ -91,6 +91,29 @@ int make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t r
   return PKV_OK;
 }
 
+// Map of a bf16 cache for the tensor-core decode kernels: 4-D (64 dims,
+// tokens, 64-dim halves, KV heads) with a box of {64, 16, D / 64, 1}, so that
+// one TMA load brings a 16-token tile as D / 64 swizzled 16 x 128 B sub-tiles.
+// The dims of one token are contiguous, so its halves lie 128 bytes apart.
+int make_stage_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t rows,
+                   pkv_dtype dtype) {
+  if (dtype != PKV_BF16 || D % 64 != 0) return PKV_ERR_UNSUPPORTED;
+  auto fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[4] = {64u, (cuuint64_t)rows, (cuuint64_t)(D / 64), (cuuint64_t)Hkv};
+  cuuint64_t strides[3] = {(cuuint64_t)Hkv * D * 2, 128u, (cuuint64_t)D * 2};
+  cuuint32_t box[4] = {64u, (cuuint32_t)pkv::kStageTokens, (cuuint32_t)(D / 64), 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {  // reported as 100000 + the driver's CUresult
+    g_last_cuda_error = 100000 + static_cast<int>(r);
+    return PKV_ERR_CUDA;
+  }
+  return PKV_OK;
+}
+
 // Raises the dynamic shared-memory limit of a kernel once per device.  `done`
 // must be distinct for every kernel (all decode kernels share one C++ type).
 template <typename Kernel>
@@ -308,14 +331,14 @@ int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap&
 #ifndef PKV_GROUP_STAGES_D128
 #define PKV_GROUP_STAGES_D128 2
 #endif
-#ifndef PKV_GROUP_WARPS
-#define PKV_GROUP_WARPS 6
+#ifndef PKV_GROUP_WARPS_D128
+#define PKV_GROUP_WARPS_D128 6
 #endif
 template <int D>
 int launch_group(const pkv::SharedParams& sp, int64_t items, const CUtensorMap& mk,
                  const CUtensorMap& mv, cudaStream_t stream) {
   constexpr int kStages = D == 128 ? PKV_GROUP_STAGES_D128 : pkv::MmaConsumer<D, 2>::kStages;
-  constexpr int W = PKV_GROUP_WARPS;
+  constexpr int W = D == 128 ? PKV_GROUP_WARPS_D128 : 6;
   using C = pkv::MmaConsumer<D, 2, kStages>;
   auto kernel = pkv::paged_decode_group_kernel<C, D, W>;
   const size_t smem = pkv::GroupSmem<C, D, W>::kBytes;
@@ -448,8 +471,12 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const bool tc = use_tensor_cores(dtype, G);
   CUtensorMap mk, mv;
   const int64_t rows = num_blocks * block_size;
-  if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, tc)) != PKV_OK) return rc;
-  if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, tc)) != PKV_OK) return rc;
+  if ((rc = tc ? make_stage_map(&mk, k_cache, D, Hkv, rows, dtype)
+                : make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, false)) != PKV_OK)
+    return rc;
+  if ((rc = tc ? make_stage_map(&mv, v_cache, D, Hkv, rows, dtype)
+                : make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, false)) != PKV_OK)
+    return rc;
 
   const bool bal = shape.balanced;
   if (tc) {
@@ -599,8 +626,8 @@ int shared_impl(void* out, const void* q, const void* k_cache, const void* v_cac
 
   CUtensorMap mk, mv;
   const int64_t rows = num_blocks * block_size;
-  if ((rc = make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
-  if ((rc = make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, true)) != PKV_OK) return rc;
+  if ((rc = make_stage_map(&mk, k_cache, D, Hkv, rows, dtype)) != PKV_OK) return rc;
+  if ((rc = make_stage_map(&mv, v_cache, D, Hkv, rows, dtype)) != PKV_OK) return rc;
   if (grouped) {
     if (D == 64) return launch_group<64>(sp, items, mk, mv, stream);
     if (D == 128) return launch_group<128>(sp, items, mk, mv, stream);

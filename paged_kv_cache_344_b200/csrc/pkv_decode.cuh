@@ -374,14 +374,13 @@ struct MmaConsumer {
     }
   }
 
+  // One box per tile: the stage maps are 4-D (64 dims, tokens, 64-dim halves,
+  // KV heads), so a box of 16 tokens lands as SUB swizzled 16 x 128 B sub-tiles.
   static __device__ __forceinline__ void load_stage(uint8_t* st, const CUtensorMap* tk,
                                                     const CUtensorMap* tv, uint64_t* bar,
                                                     int kvh, int row, uint64_t pol) {
-#pragma unroll
-    for (int sb = 0; sb < SUB; ++sb) {
-      tma_load_3d(st + sb * kSubBytes, tk, bar, sb * 64, kvh, row, pol);
-      tma_load_3d(st + kTileBytes + sb * kSubBytes, tv, bar, sb * 64, kvh, row, pol);
-    }
+    tma_load_4d(st, tk, bar, 0, row, 0, kvh, pol);
+    tma_load_4d(st + kTileBytes, tv, bar, 0, row, 0, kvh, pol);
   }
 
   // Byte offset of (row, 16-byte chunk) inside a swizzled 16x128 B sub-tile.
@@ -410,12 +409,13 @@ struct MmaConsumer {
     // state is what a fully masked stage would leave.
     auto live = [&](int nt) { return !kRows || (nt * 8 < r1 && nt * 8 + 8 > r0); };
 
-    // Scores: S = K Q^T, one m16n8k16 per (k-step, head tile).
-    float s[NT][4];
+    // Scores: S = K Q^T, one m16n8k16 per (k-step, head tile), the even and
+    // the odd k-steps in two accumulators so that the MMA chain is half as long.
+    float s[NT][4], s2[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) s[nt][j] = 0.f;
+      for (int j = 0; j < 4; ++j) s[nt][j] = s2[nt][j] = 0.f;
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       const int row = rr + (mi & 1) * 8;
@@ -424,8 +424,12 @@ struct MmaConsumer {
       ldmatrix_x4(sk + (ks / 4) * kSubBytes + swz(row, chunk), a[0], a[1], a[2], a[3]);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
-        if (live(nt)) mma_bf16_16816(s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
+        if (live(nt)) mma_bf16_16816(ks % 2 ? s2[nt] : s[nt], a, qf[nt][ks][0], qf[nt][ks][1]);
     }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) s[nt][j] += s2[nt][j];
 
     // Invalid tail slots of the last stage hold anything (even NaN): their
     // scores are replaced by -inf, and their V rows are zeroed before the PV

@@ -339,14 +339,25 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
 // masked).  The warps take stages round-robin, so each warp's running softmax
 // state covers some prefix stages and some own stages; merging the warps gives
 // every row exactly its prefix plus its own tokens.  No partials leave the CTA.
+// Shared memory of a group CTA: one slot per warp that holds its ring of
+// stages and, at the end, its softmax state (M, l and O of 16 rows) for the
+// merge; slots start on 1024-byte boundaries (the swizzled TMA boxes need it).
+template <class C, int D, int W>
+struct GroupSmem {
+  static constexpr int kStateBytes = (2 * C::GP + C::GP * D) * 4;
+  static constexpr int kRingBytes = DecodeSmem<C>::kRingBytes;
+  static constexpr int kSlot =
+      ((kRingBytes > kStateBytes ? kRingBytes : kStateBytes) + 1023) / 1024 * 1024;
+  static constexpr size_t kBytes = 1024 /*alignment slack*/ + (size_t)W * kSlot + W * C::kStages * 8;
+};
+
 template <class C, int D, int W>
 __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kvh, uint8_t* smem,
                                             const CUtensorMap& tmK, const CUtensorMap& tmV) {
   using T = __nv_bfloat16;
-  constexpr int kRing = DecodeSmem<C>::kRingBytes;
+  constexpr int kRing = GroupSmem<C, D, W>::kSlot;  // stride of the warps' slots
   constexpr int kMaxMembers = 16;
   static_assert(C::GP == 16, "group pieces use the 16-row consumer");
-  static_assert(kRing >= (2 * C::GP + C::GP * D) * 4, "state does not fit in the ring");
   __shared__ int s_len[kMaxMembers], s_cum[kMaxMembers + 1];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * kRing);
   const DecodeParams& p = s.d;
@@ -391,23 +402,20 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     }
   }
   const int n_pre = s_cum[0], n_all = s_cum[members];
-  // Stage k of the CTA: table row, first token, valid tokens, rows that score it.
-  auto stage_of = [&](int k, int& b, int& t0, int& nv, int& r0, int& r1) {
+  // Stage k of the CTA: the member i whose table row it reads, its first token
+  // and its valid tokens; true when every member's rows score it (a prefix stage,
+  // or any stage of a one-member group), else only member i's rows do.
+  auto stage_of = [&](int k, int& i, int& t0, int& nv) -> bool {
+    i = 0;
     if (k < n_pre) {
-      b = lo;
       t0 = k * kStageTokens;
       nv = kStageTokens;
-      r0 = 0;
-      r1 = members * G;
-      return;
+      return true;
     }
-    int i = 0;
     while (k >= s_cum[i + 1]) ++i;
-    b = lo + i;
     t0 = plen + (k - s_cum[i]) * kStageTokens;
     nv = min(kStageTokens, s_len[i] - t0);
-    r0 = i * G;
-    r1 = r0 + G;
+    return members == 1;
   };
   // This warp takes the CTA's stages warp, warp + W, ...
   const int first = warp, stride = W;
@@ -423,35 +431,42 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   }
   __syncwarp();
   const uint64_t pol = l2_policy_evict_first();
-  auto stage_id = [&](int kk) -> int {  // block id of the warp's kk-th stage
-    int b, t0, nv, r0, r1;
-    stage_of(first + stride * kk, b, t0, nv, r0, r1);
-    return p.block_tables[(size_t)b * p.max_blocks + t0 / p.bs];
+  // The warp's stages win_base .. win_base + 63 are resolved ahead, one per lane
+  // of two windows: the TMA row of the stage's 16 tokens (past the pool, so
+  // that TMA fills zeros, for a block id out of range) and its meta word (valid
+  // tokens | member << 5 | every-row flag << 10).  Lane 0 files the meta word of
+  // each stage it loads in s_meta beside the stage's slot.
+  __shared__ int s_meta[W][C::kStages];
+  auto stage_info = [&](int kk, int& meta) -> int {
+    int i, t0, nv;
+    const bool all_rows = stage_of(first + stride * kk, i, t0, nv);
+    meta = nv | (i << 5) | (all_rows ? 1 << 10 : 0);
+    const int id = p.block_tables[(size_t)(lo + i) * p.max_blocks + t0 / p.bs];
+    if (id < 0 || id >= p.num_blocks) {
+      flag_error(PKV_DEVERR_BLOCK_ID);
+      return p.num_blocks * p.bs;
+    }
+    return id * p.bs + t0 % p.bs;
   };
-  int win_base = 0;
-  int win0 = lane < n_w ? stage_id(lane) : -1;
-  int win1 = 32 + lane < n_w ? stage_id(32 + lane) : -1;
+  int win_base = 0, wm0 = 0, wm1 = 0;
+  int win0 = lane < n_w ? stage_info(lane, wm0) : 0;
+  int win1 = 32 + lane < n_w ? stage_info(32 + lane, wm1) : 0;
   auto issue = [&](int kk) {
     if (kk - win_base >= 32) {
       win0 = win1;
+      wm0 = wm1;
       win_base += 32;
-      win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane) : -1;
+      win1 = win_base + 32 + lane < n_w ? stage_info(win_base + 32 + lane, wm1) : 0;
     }
-    const int id = __shfl_sync(kFull, win0, kk - win_base);  // kk - win_base < 32 here
+    const int row = __shfl_sync(kFull, win0, kk - win_base);  // kk - win_base < 32 here
+    const int meta = __shfl_sync(kFull, wm0, kk - win_base);
     if (lane == 0) {
-      int b, t0, nv, r0, r1;
-      stage_of(first + stride * kk, b, t0, nv, r0, r1);
       const int st = kk % C::kStages;
-      int row;
-      if (id < 0 || id >= p.num_blocks) {
-        flag_error(PKV_DEVERR_BLOCK_ID);
-        row = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
-      } else {
-        row = id * p.bs + t0 % p.bs;
-      }
+      s_meta[warp][st] = meta;
       mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
       C::load_stage(ring + st * C::kStageBytes, &tmK, &tmV, &wbar[st], kvh, row, pol);
     }
+    __syncwarp();  // the meta word is seen by every lane before the stage is consumed
   };
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
   for (int kk = 0; kk < n_pro; ++kk) issue(kk);
@@ -467,49 +482,71 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
         mbar_wait_bounded(&wbar[j % C::kStages], (uint32_t)((j / C::kStages) & 1));
       break;
     }
-    int b, t0, nv, r0, r1;
-    stage_of(first + stride * kk, b, t0, nv, r0, r1);
-    if (r0 == 0 && r1 == members * G)  // a prefix stage: every member's rows
+    const int meta = s_meta[warp][st];
+    const int nv = meta & 31, r0 = ((meta >> 5) & 31) * G;
+    if (meta >> 10)  // every member's rows score it
       c.consume(ring + st * C::kStageBytes, nv, lane);
     else
-      c.consume_rows(ring + st * C::kStageBytes, nv, lane, r0, r1);
+      c.consume_rows(ring + st * C::kStageBytes, nv, lane, r0, r0 + G);
     __syncwarp();
     if (kk + C::kStages < n_w) issue(kk + C::kStages);
   }
 
-  // Merge the warps; each row n = member * G + head goes to its sequence.  A row
-  // with no token at all (an empty sequence) is written as zeros.
+  // Merge the warps; each row n = member * G + head goes to its sequence.  The
+  // weights exp2(m_w - M) of each (warp, row) and 1 / l of each row are formed
+  // once, then every thread combines 8 consecutive dims of one row.  A row with
+  // no token at all (an empty sequence) is written as zeros.
   c.store_state(reinterpret_cast<float*>(ring), lane);
   __syncthreads();
   constexpr int GP = C::GP;
+  __shared__ float s_wt[W][GP], s_inv[GP];
+  auto state = [&](int w) { return reinterpret_cast<const float*>(smem + w * kRing); };
   const int rows = members * G;
-  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
-    const int n = idx / D, d = idx % D;
+  if (threadIdx.x < rows) {
+    const int n = threadIdx.x;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < W; ++w) M = fmaxf(M, reinterpret_cast<const float*>(smem + w * kRing)[n]);
-    float num = 0.f, den = 0.f;
-    if (M != -INFINITY) {
+    for (int w = 0; w < W; ++w) M = fmaxf(M, state(w)[n]);
+    float den = 0.f;
 #pragma unroll
-      for (int w = 0; w < W; ++w) {
-        const float* stt = reinterpret_cast<const float*>(smem + w * kRing);
-        const float f = exp2f(stt[n] - M);
-        num = fmaf(f, stt[2 * GP + n * D + d], num);
-        den = fmaf(f, stt[GP + n], den);
-      }
+    for (int w = 0; w < W; ++w) {
+      const float f = M == -INFINITY ? 0.f : exp2f(state(w)[n] - M);
+      s_wt[w][n] = f;
+      den = fmaf(f, state(w)[GP + n], den);
     }
-    out[((size_t)(lo + n / G) * p.Hq + (size_t)kvh * G + n % G) * D + d] =
-        __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+    s_inv[n] = den > 0.f ? 1.f / den : 0.f;
+  }
+  __syncthreads();
+  constexpr int kChunks = D / 8;
+  for (int idx = threadIdx.x; idx < rows * kChunks; idx += blockDim.x) {
+    const int n = idx / kChunks, d0 = (idx % kChunks) * 8;
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w = 0; w < W; ++w) {
+      const float f = s_wt[w][n];
+      const float4* src = reinterpret_cast<const float4*>(state(w) + 2 * GP + n * D + d0);
+      const float4 x = src[0], y = src[1];
+      a[0] = fmaf(f, x.x, a[0]);
+      a[1] = fmaf(f, x.y, a[1]);
+      a[2] = fmaf(f, x.z, a[2]);
+      a[3] = fmaf(f, x.w, a[3]);
+      a[4] = fmaf(f, y.x, a[4]);
+      a[5] = fmaf(f, y.y, a[5]);
+      a[6] = fmaf(f, y.z, a[6]);
+      a[7] = fmaf(f, y.w, a[7]);
+    }
+    const float inv = s_inv[n];
+    uint4 v;
+    v.x = pack_bf16x2(a[0] * inv, a[1] * inv);
+    v.y = pack_bf16x2(a[2] * inv, a[3] * inv);
+    v.z = pack_bf16x2(a[4] * inv, a[5] * inv);
+    v.w = pack_bf16x2(a[6] * inv, a[7] * inv);
+    *reinterpret_cast<uint4*>(out + ((size_t)(lo + n / G) * p.Hq + (size_t)kvh * G + n % G) * D +
+                              d0) = v;
   }
 }
 
 // One CTA of W warps per (group, KV head): group_piece with consumer C (16 rows).
-template <class C, int D, int W>
-struct GroupSmem {
-  static constexpr size_t kBytes =
-      1024 /*alignment slack*/ + (size_t)W * DecodeSmem<C>::kRingBytes + W * C::kStages * 8;
-};
-
 template <class C, int D, int W>
 __global__ void __launch_bounds__(W * 32)
     paged_decode_group_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
