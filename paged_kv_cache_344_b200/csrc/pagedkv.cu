@@ -325,9 +325,11 @@ int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap&
 }
 
 // One CTA of GROUP_WARPS warps per (group, KV head), 16-row consumer with a
-// ring of GROUP_STAGES stages per warp.  Measured on B200 (share workloads):
-// 6 warps (2 CTAs per SM) beat 4 by up to 7% and 8 (1 CTA per SM) are 1.3x
-// slower; 3 stages equal 2, 4 stages (1 CTA per SM) are 1.6x slower.
+// ring of GROUP_STAGES stages per warp (D = 128; other head dims: 6 warps and
+// the consumer's default ring).  Measured on B200 (share workloads): 6 warps
+// (2 CTAs per SM) beat 4 by up to 7% and 8 (1 CTA per SM) are 1.3x slower;
+// 3 stages equal 2, 4 stages (1 CTA per SM) are 1.6x slower.  At 160 registers
+// a thread two CTAs of 6 warps fill an SM's register file.
 #ifndef PKV_GROUP_STAGES_D128
 #define PKV_GROUP_STAGES_D128 2
 #endif
