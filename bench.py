@@ -65,7 +65,12 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {"decode": ("pkv_ptx.cuh", "pkv_decode.cuh"),
+                  "shared": ("pkv_ptx.cuh", "pkv_decode.cuh", "pkv_decode_shared.cuh"),
                   "prefill": ("pkv_ptx.cuh", "pkv_decode.cuh", "pkv_prefill.cuh")}
+
+# Decode workloads of the benchmark definition reported beside the headline, each timed
+# the same way (``per_config``).
+PER_CONFIG = ["mha", "gqa16", "gqa32", "long", "share_fork", "share_tails"]
 
 
 def kernel_source_sha(kind: str = "decode") -> str:
@@ -81,7 +86,8 @@ def kernel_source_sha(kind: str = "decode") -> str:
 def recorded_traffic(config: str, partition: int, kind: str = "decode"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel sources (and, for decode, the same partition length); else None."""
-    path = os.path.join(ROOT, "profiles", f"{kind}_{config}_ncu.md")
+    prefix = "prefill" if kind == "prefill" else "decode"
+    path = os.path.join(ROOT, "profiles", f"{prefix}_{config}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
@@ -90,7 +96,7 @@ def recorded_traffic(config: str, partition: int, kind: str = "decode"):
     q = re.search(r"partition_tokens:\s*([0-9]+)", text)
     if not m or not s or s.group(1) != kernel_source_sha(kind):
         return None
-    if kind == "decode" and (not q or int(q.group(1)) != partition):
+    if kind in ("decode", "shared") and (not q or int(q.group(1)) != partition):
         return None
     return float(m.group(1))
 
@@ -191,56 +197,83 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------
 # CPU side: the oracle on a bounded sample
 # ----------------------------------------------------------------------------------------
-def oracle_sample(wl, host_pool, budget_rows: int):
-    """Sequences 0..n-1 whose rows stay under ``budget_rows`` row-tokens; returns the oracle
-    inputs for them and their algorithmic bytes."""
-    lens = wl.seq_lens_post
+def oracle_sample_size(wl, budget_rows: int) -> int:
+    """Sequences 0..n-1 whose query-row x token work stays under ``budget_rows``."""
     acc, n = 0, 0
     for b in range(wl.B):
-        acc += int(lens[b]) * wl.Hq
+        acc += int(wl.seq_lens_post[b]) * wl.Hq
         n = b + 1
         if acc >= budget_rows:
             break
     return n
 
 
-def time_oracle(wl, host, n_seq: int):
+def sample_bytes(wl, sample) -> int:
+    """Algorithmic bytes of the sample's decode (its distinct blocks once, q, out, tables)."""
+    nb = sample["k_cache"].shape[0]
+    n = sample["q"].shape[0]
+    tables = sum(-(-int(L) // wl.bs) for L in sample["seq_lens"])
+    return int(nb * wl.block_bytes * 2 + 2 * n * wl.Hq * wl.D * wl.elt + tables * 4 + 4 * n)
+
+
+def time_oracle(wl, sample):
+    """Seconds of one fp64 oracle decode of the sample, its bytes, tokens and threads."""
     import oracle
-    q = np.ascontiguousarray(host["q"][:n_seq])
-    bt = np.ascontiguousarray(wl.block_tables[:n_seq])
-    sl = np.ascontiguousarray(wl.seq_lens_post[:n_seq])
     t0 = time.perf_counter()
-    oracle.paged_decode(q, host["k_cache"], host["v_cache"], bt, sl, wl.scale)
+    oracle.paged_decode(sample["q"], sample["k_cache"], sample["v_cache"],
+                        sample["block_tables"], sample["seq_lens"], wl.scale)
     dt = time.perf_counter() - t0
-    blocks = sum(-(-int(L) // wl.bs) for L in sl)
-    nbytes = blocks * wl.block_bytes * 2 + 2 * n_seq * wl.Hq * wl.D * wl.elt + blocks * 4
-    return dt, nbytes, int(sl.sum()), oracle.num_threads()
+    return dt, sample_bytes(wl, sample), int(sample["seq_lens"].sum()), oracle.num_threads()
 
 
-def host_pool_from(dev, wl):
+def cpu_baseline_of(wl, dev, budget_rows: int):
+    """The oracle on sequences 0..n-1 of the workload, over their blocks gathered from the
+    device pool after the step (so the sample is the step's own post-step state)."""
     import torch
-    out = {}
-    for k in ("q", "k_cache", "v_cache"):
-        t = dev[k].detach().cpu().contiguous()
-        out[k] = t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
-    return out
+    n_seq = oracle_sample_size(wl, budget_rows)
+    sample = workloads.compact_sample(wl, n_seq, dev["k_cache"], dev["v_cache"])
+    q = dev["q"][:n_seq].detach().cpu().contiguous()
+    sample["q"] = q.view(torch.int16).numpy().view(np.uint16) if q.dtype == torch.bfloat16 \
+        else q.numpy()
+    dt, nbytes, tokens, cores = time_oracle(wl, sample)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"decode of sequences 0..{n_seq - 1} of {wl.B} ({tokens} cached tokens, "
+                      f"{n_seq * wl.Hq} query rows, {sample['k_cache'].shape[0]} distinct blocks),"
+                      f" fp64, {dt:.2f} s",
+            "tokens_per_s": round(n_seq / dt, 3)}
 
 
 # ----------------------------------------------------------------------------------------
 # GPU side
 # ----------------------------------------------------------------------------------------
-def run_ours(args, rank, world, local_rank):
+def config_dict(args, name, wl, fused: bool, use_shared: bool, has_cow: bool, world: int):
+    """The workload's description; both arms report the same dict."""
+    step_bytes = (workloads.decode_algorithmic_bytes(wl) + workloads.write_bytes(wl) +
+                  workloads.copy_bytes(wl))
+    working_set = workloads.decode_algorithmic_bytes(wl)
+    flush = working_set < 8 * L2_BYTES
+    entry = "paged_attention_decode_shared_prefix" if use_shared else "paged_attention_decode"
+    return {"workload": name, "description": DESCR.get(name, name),
+            "step": (("paged_decode_step_shared_prefix" if use_shared else "paged_decode_step")
+                     + " (copy-on-write + cache write + decode in one launch)" if fused else
+                     ("copy_blocks + " if has_cow else "") + "paged_kv_write + " + entry),
+            "bytes_per_step": step_bytes,
+            "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
+                   else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "block_size": wl.bs, "placement": "contiguous" if args.contiguous else "shuffled"}
+
+
+def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, with_cpu):
+    """One workload: warm-up, ``steps`` timed decode steps (device events on the launching
+    stream), optionally the end-to-end pipelined measurement and the oracle baseline."""
     import torch
     import torch.distributed as dist
     import paged_kv_cache_344_b200 as pkv
 
-    torch.cuda.set_device(local_rank)
     dev_name = f"cuda:{local_rank}"
-    pkv.set_decode_path({"auto": pkv.PKV_PATH_AUTO, "cuda_cores": pkv.PKV_PATH_CUDA_CORES,
-                         "tensor_cores": pkv.PKV_PATH_TENSOR_CORES}[args.path])
-    pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED if args.split == "balanced" else pkv.PKV_SPLIT_FIXED)
-    wl = workloads.make(args.config, block_size=args.block_size or None,
-                        contiguous=args.contiguous)
+    wl = workloads.make(name, block_size=args.block_size or None, contiguous=args.contiguous)
     dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
     meta = {
         "block_tables": torch.from_numpy(wl.block_tables).to(dev_name),
@@ -249,7 +282,7 @@ def run_ours(args, rank, world, local_rank):
         "cow_pairs": torch.from_numpy(wl.cow_pairs).to(dev_name),
     }
     use_shared = args.decode == "shared_prefix" or (args.decode == "auto"
-                                                    and args.config.startswith("share"))
+                                                    and name.startswith("share"))
     if use_shared:
         ws_bytes = pkv.paged_attention_decode_shared_prefix_workspace_size(
             wl.B, wl.Hq, wl.Hkv, wl.D, wl.max_seq_len, wl.bs, args.partition)
@@ -313,11 +346,10 @@ def run_ours(args, rank, world, local_rank):
 
     d_in = dict(dev)
     d_in.update(meta)
-    step_bytes = (workloads.decode_algorithmic_bytes(wl) + workloads.write_bytes(wl) +
-                  workloads.copy_bytes(wl))
+    cfg = config_dict(args, name, wl, fused, use_shared, has_cow, world)
+    step_bytes = cfg["bytes_per_step"]
     decode_bytes = workloads.decode_algorithmic_bytes(wl)
-    working_set = decode_bytes
-    flush = working_set < 8 * L2_BYTES
+    flush = decode_bytes < 8 * L2_BYTES
     scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev_name) if flush else None
 
     def barrier():
@@ -325,7 +357,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step(d_in)
     if flush:
         scratch.fill_(1)
@@ -333,16 +365,16 @@ def run_ours(args, rank, world, local_rank):
 
     def timed_region():
         ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
+                  for _ in range(steps)]
         ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
+                   for _ in range(steps)]
         barrier()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         with ClockSampler(local_rank) as clocks:
             torch.cuda.nvtx.range_push("timed_region")
             t_start.record(stream)
-            for i in range(args.steps):
+            for i in range(steps):
                 if flush:
                     scratch.add_(1)  # evict the previous step's blocks from L2 (untimed below)
                 ev_step[i][0].record(stream)
@@ -364,14 +396,56 @@ def run_ours(args, rank, world, local_rank):
 
     # max over ranks (device-timed)
     total_ms_max = max_over_ranks(total_ms, world, dev_name)
-    ms_per_step = total_ms_max / args.steps
-    value = whole_job_gbs(step_bytes, args.steps, world, total_ms_max)
-    tokens_per_s = world * wl.B * args.steps / (total_ms_max * 1e-3)
+    ms_per_step = total_ms_max / steps
+    value = whole_job_gbs(step_bytes, steps, world, total_ms_max)
+    tokens_per_s = world * wl.B * steps / (total_ms_max * 1e-3)
 
-    # e2e through the public API: every step copies its inputs from pinned host memory and
-    # reads its output back.  As in a serving loop, the copies of step i+1's inputs and of
-    # step i's output run on a copy stream and overlap the computation of step i (two sets
-    # of step buffers; the KV cache itself stays resident).
+    peak, peak_src = load_peaks()
+    dec_avg_ms = statistics.fmean(dec_ms)
+    kernel_bytes = step_bytes if fused else decode_bytes  # the fused kernel also writes/copies
+    achieved = kernel_bytes / (dec_avg_ms * 1e-3) / 1e9
+    tc = wl.dtype == "bf16" and (args.path != "cuda_cores" or wl.G > 8)
+    grouped = use_shared and args.partition == 0 and int(np.diff(wl.group_offsets).max()) <= \
+        max(1, 16 // wl.G)
+    kernel = ("paged_decode_group_kernel" if grouped else
+              "paged_decode_shared_kernel" if use_shared else
+              "paged_decode_kernel" if fused else
+              "paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
+        + ("<MmaConsumer>" if tc else "<SimtConsumer>")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4),
+                "traffic": recorded_traffic(name, part, "shared" if use_shared else "decode"),
+                "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
+                "decode_us": round(dec_avg_ms * 1e3, 2),
+                "algorithmic_bytes_per_launch": kernel_bytes,
+                "achieved_token_exact": round(workloads.decode_token_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9, 1)}
+    res = {"value": round(value, 1), "ms_per_step": round(ms_per_step, 5),
+           "tokens_per_s": round(tokens_per_s, 1), "config": cfg,
+           "launch": {"decode_entry": "paged_attention_decode_shared_prefix" if use_shared
+                      else "paged_attention_decode", "decode_path": args.path,
+                      "decode_split": args.split, "partition_tokens": part},
+           "roofline": roofline, "gpu_launches": launches_per_step * steps,
+           "clocks": clocks.summary(), "dtype": wl.dtype}
+    if remeasured:
+        res["clocks"]["remeasured"] = True
+
+    if with_e2e:
+        res["e2e"] = run_e2e(step, d_in, out, has_cow, stream, step_bytes, wl, world, dev_name,
+                             steps, warmup, barrier)
+    res["cpu_baseline"] = None
+    if with_cpu and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_of(wl, dev, args.cpu_budget_rows)
+    return res
+
+
+def run_e2e(step, d_in, out, has_cow, stream, step_bytes, wl, world, dev_name, steps, warmup,
+            barrier):
+    """e2e through the public API: every step copies its inputs from pinned host memory and
+    reads its output back.  As in a serving loop, the copies of step i+1's inputs and of
+    step i's output run on a copy stream and overlap the computation of step i (two sets
+    of step buffers; the KV cache itself stays resident)."""
+    import torch
     in_keys = [k for k in ("q", "k_new", "v_new", "block_tables", "seq_lens", "slot_mapping",
                            "cow_pairs", "group_offsets", "prefix_lens", "cow_src")
                if k in d_in and (k != "cow_pairs" or has_cow)]
@@ -418,81 +492,62 @@ def run_ours(args, rank, world, local_rank):
             comp_(i)
             d2h_(i)
 
-    e2e_run(max(3, args.warmup // 4))
+    e2e_run(max(3, warmup // 4))
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_steps = max(10, args.steps // 4)
+    e2e_steps = max(10, steps // 4)
     e0.record(copy_s)
     e2e_run(e2e_steps)
     e1.record(copy_s)
     barrier()
     e2e_ms_max = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev_name)
-    e2e_val = whole_job_gbs(step_bytes, 1, world, e2e_ms_max)
+    return {"value": round(whole_job_gbs(step_bytes, 1, world, e2e_ms_max), 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(e2e_ms_max, 5),
+            "tokens_per_s": round(world * wl.B / (e2e_ms_max * 1e-3), 1),
+            "pipelining": "inputs of step i+1 and output of step i copied on a second "
+                          "stream while step i computes"}
 
-    peak, peak_src = load_peaks()
-    dec_avg_ms = statistics.fmean(dec_ms)
-    kernel_bytes = step_bytes if fused else decode_bytes  # the fused kernel also writes/copies
-    achieved = kernel_bytes / (dec_avg_ms * 1e-3) / 1e9
-    G = wl.G
-    tc = wl.dtype == "bf16" and (args.path != "cuda_cores" or G > 8)
-    kernel = ("paged_decode_shared_kernel" if use_shared else
-              "paged_decode_kernel" if fused else
-              "paged_decode_balanced_kernel" if args.split == "balanced" else "paged_decode_kernel") \
-        + ("<MmaConsumer>" if tc else "<SimtConsumer>")
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": recorded_traffic(args.config, part),
-                "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
-                "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
-                "decode_us": round(dec_avg_ms * 1e3, 2),
-                "algorithmic_bytes_per_launch": kernel_bytes,
-                "achieved_token_exact": round(workloads.decode_token_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9, 1)}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = host_pool_from(dev, wl)
-        n_seq = oracle_sample(wl, host, budget_rows=args.cpu_budget_rows)
-        dt, nbytes, tokens, cores = time_oracle(wl, host, n_seq)
-        cpu = {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
-               "kind": "oracle",
-               "sample": f"decode of sequences 0..{n_seq - 1} of {wl.B} ({tokens} cached tokens, "
-                         f"{n_seq * wl.Hq} query rows), fp64, {dt:.2f} s",
-               "tokens_per_s": round(n_seq / dt, 3)}
+def run_ours(args, rank, world, local_rank):
+    """The headline workload with its e2e and oracle legs, then every other decode workload
+    of the benchmark definition as a ``per_config`` entry."""
+    import torch
+    import paged_kv_cache_344_b200 as pkv
 
+    torch.cuda.set_device(local_rank)
+    pkv.set_decode_path({"auto": pkv.PKV_PATH_AUTO, "cuda_cores": pkv.PKV_PATH_CUDA_CORES,
+                         "tensor_cores": pkv.PKV_PATH_TENSOR_CORES}[args.path])
+    pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED if args.split == "balanced" else pkv.PKV_SPLIT_FIXED)
+    head = run_decode(args, args.config, rank, world, local_rank, args.steps, args.warmup,
+                      with_e2e=True, with_cpu=True)
+    peak = head["roofline"]["peak"]
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
         "data": "synthetic (seeded N(0,1) q/K/V, shuffled block pool, NaN in unused slots)",
-        "tokens_per_s": round(tokens_per_s, 1),
-        "pct_of_8TBps_spec": round(100 * value / world / SPEC_HBM_GBS, 2),
-        "pct_of_measured_peak": round(100 * value / world / peak, 2),
-        "config": {"workload": args.config, "description": DESCR.get(args.config, args.config),
-                   "step": (("paged_decode_step_shared_prefix" if use_shared else "paged_decode_step")
-                            + " (copy-on-write + cache write + decode in one launch)" if fused else
-                            ("copy_blocks + " if has_cow else "") + "paged_kv_write + "
-                            + ("paged_attention_decode_shared_prefix" if use_shared
-                               else "paged_attention_decode")),
-                   "bytes_per_step": step_bytes,
-                   "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
-                          else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "decode_entry": "paged_attention_decode_shared_prefix" if use_shared
-                   else "paged_attention_decode",
-                   "block_size": wl.bs, "placement": "contiguous" if args.contiguous else "shuffled",
-                   "decode_path": args.path, "decode_split": args.split,
-                   "partition_tokens": part},
-        "roofline": roofline,
-        "cpu_baseline": cpu,
-        "e2e": {"value": round(e2e_val, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms_max, 5),
-                "tokens_per_s": round(world * wl.B / (e2e_ms_max * 1e-3), 1),
-                "pipelining": "inputs of step i+1 and output of step i copied on a second "
-                              "stream while step i computes"},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clocks.summary(),
+        "tokens_per_s": head["tokens_per_s"],
+        "pct_of_8TBps_spec": round(100 * head["value"] / world / SPEC_HBM_GBS, 2),
+        "pct_of_measured_peak": round(100 * head["value"] / world / peak, 2),
+        "config": head["config"], "launch": head["launch"], "roofline": head["roofline"],
+        "cpu_baseline": head["cpu_baseline"], "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
     }
-    if remeasured:
-        line["clocks"]["remeasured"] = True
+    if not args.no_per_config:
+        per = {}
+        for name in PER_CONFIG:
+            if name == args.config:
+                continue
+            torch.cuda.empty_cache()
+            r = run_decode(args, name, rank, world, local_rank, args.steps, args.warmup,
+                           with_e2e=False, with_cpu=True)
+            per[name] = {"value": r["value"], "unit": "GB/s", "ms_per_step": r["ms_per_step"],
+                         "tokens_per_s": r["tokens_per_s"], "config": r["config"],
+                         "launch": r["launch"], "roofline": r["roofline"],
+                         "cpu_baseline": r["cpu_baseline"], "gpu_launches": r["gpu_launches"],
+                         "clocks": r["clocks"]}
+        line["per_config"] = per
     return line
 
 
@@ -623,6 +678,103 @@ def run_prefill(args, rank, world, local_rank):
             "clocks": clocks.summary()}
 
 
+def run_paging(args, local_rank):
+    """The paging-overhead control and the block-size sweep ([Index] "Limitations": the
+    block-table walk may cost a little against a contiguous allocation; [Explained] "2.
+    Partial Block Waste": block size trades wasted slots against management overhead).
+    For each workload: the decode alone (CUDA events on its stream) over the shuffled pool,
+    over a pool whose blocks are laid out in order, with the table-free kernel on the same
+    logical K/V as the shuffled pool, and over shuffled pools of 8/16/32/64-token blocks."""
+    import torch
+    import paged_kv_cache_344_b200 as pkv
+    torch.cuda.set_device(local_rank)
+    dev_name = f"cuda:{local_rank}"
+    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev_name)
+
+    def time_decode(fn, nbytes):
+        flush = nbytes < 8 * L2_BYTES
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for a, b in ev:
+            if flush:
+                scratch.add_(1)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return statistics.median(x.elapsed_time(y) for x, y in ev) * 1e3
+
+    def paged(name, **kw):
+        wl = workloads.make(name, **kw)
+        dev = workloads.device_tensors(wl, dev_name)
+        bt = torch.from_numpy(wl.block_tables).to(dev_name)
+        sl = torch.from_numpy(wl.seq_lens_post).to(dev_name)
+        n = pkv.paged_attention_decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D, wl.max_seq_len,
+                                                      wl.bs, 0)
+        ws = torch.zeros(max(n, 1), dtype=torch.uint8, device=dev_name)
+        out = torch.empty_like(dev["q"])
+
+        def fn():
+            pkv.paged_attention_decode(out, dev["q"], dev["k_cache"], dev["v_cache"], bt, sl,
+                                       wl.max_seq_len, wl.scale, workspace=ws)
+        return wl, dev, ws, fn
+
+    res = {}
+    for name in args.paging_configs.split(","):
+        r = {}
+        wl, dev, ws, fn = paged(name)
+        r["bytes_per_call"] = workloads.decode_algorithmic_bytes(wl)
+        r["token_bytes_per_call"] = workloads.decode_token_bytes(wl)
+        r["shuffled_us"] = round(time_decode(fn, r["bytes_per_call"]), 2)
+        # the same logical K/V, unpaged: [B, stride, Hkv, D] and no table at all
+        stride = wl.max_seq_len
+        cont = []
+        for key in ("k_cache", "v_cache"):
+            c = torch.zeros((wl.B, stride, wl.Hkv, wl.D), dtype=dev[key].dtype, device=dev_name)
+            for b in range(wl.B):
+                L = int(wl.seq_lens_post[b])
+                nb = -(-L // wl.bs)
+                ids = torch.from_numpy(wl.block_tables[b, :nb].astype(np.int64)).to(dev_name)
+                c[b, :L] = dev[key][ids].reshape(nb * wl.bs, wl.Hkv, wl.D)[:L]
+            cont.append(c)
+        del dev
+        torch.cuda.empty_cache()
+        q = torch.randn((wl.B, wl.Hq, wl.D), device=dev_name).to(cont[0].dtype)
+        out = torch.empty_like(q)
+        sl = torch.from_numpy(wl.seq_lens_post).to(dev_name)
+
+        def fn_c():
+            pkv.paged_attention_decode_contiguous(out, q, cont[0], cont[1], sl, wl.max_seq_len,
+                                                  wl.scale, workspace=ws)
+        r["table_free_us"] = round(time_decode(fn_c, r["bytes_per_call"]), 2)
+        del cont
+        torch.cuda.empty_cache()
+        _, _, _, fn_o = paged(name, contiguous=True)
+        r["in_order_pool_us"] = round(time_decode(fn_o, r["bytes_per_call"]), 2)
+        torch.cuda.empty_cache()
+        r["paging_overhead_vs_table_free"] = round(r["shuffled_us"] / r["table_free_us"] - 1, 4)
+        sweep = {}
+        for bs in (8, 16, 32, 64):
+            wlb, devb, _, fnb = paged(name, block_size=bs)
+            nbytes = workloads.decode_algorithmic_bytes(wlb)
+            us = time_decode(fnb, nbytes)
+            sweep[str(bs)] = {"decode_us": round(us, 2), "algorithmic_bytes": nbytes,
+                              "GBs": round(nbytes / (us * 1e-6) / 1e9, 1),
+                              "GBs_token_exact": round(workloads.decode_token_bytes(wlb) /
+                                                       (us * 1e-6) / 1e9, 1),
+                              "unused_slot_fraction": round(
+                                  1 - workloads.decode_token_bytes(wlb) / nbytes, 4)}
+            del devb
+            torch.cuda.empty_cache()
+        r["block_size_sweep"] = sweep
+        res[name] = r
+    return {"metric": "paging overhead (table-free control) and block-size sweep: decode us",
+            "unit": "us", "steps": args.steps, "warmup": args.warmup, "per_config": res}
+
+
 def prefill_oracle_sample(wl, cu_q, dev, q, budget_flops: float):
     """The fp64 oracle's multi-query attention on sequences 0..n-1 (cumulative causal flops
     up to ``budget_flops``), over a compact host pool of just their blocks; returns
@@ -662,31 +814,37 @@ def prefill_oracle_sample(wl, cu_q, dev, q, budget_flops: float):
 
 def run_reference(args, rank, world):
     """The reference arm: the fp64 oracle on this host's cores, each step a bounded sample
-    of the same workload."""
+    of the same workload (the blocks of its first sequences, drawn on the host)."""
     if rank != 0:
         return None
-    wl = workloads.make(args.config)
-    host = workloads.host_tensors(wl) if wl.num_blocks * wl.block_bytes < (6 << 30) else None
-    if host is None:
-        raise SystemExit("workload too large for a host-side reference run")
-    n_seq = oracle_sample(wl, host, budget_rows=args.cpu_budget_rows // max(args.steps, 1))
+    wl = workloads.make(args.config, block_size=args.block_size or None,
+                        contiguous=args.contiguous)
+    n_seq = oracle_sample_size(wl, args.cpu_budget_rows // max(args.steps, 1))
+    sample = workloads.compact_sample(wl, n_seq)
+    nw = max(1, n_seq // 8)  # warm-up: the first sequences of the same sample
+    warm = dict(sample, q=sample["q"][:nw], block_tables=sample["block_tables"][:nw],
+                seq_lens=sample["seq_lens"][:nw])
     for _ in range(args.warmup):
-        time_oracle(wl, host, max(1, n_seq // 8))
-    total_t, total_b, cores, tokens = 0.0, 0, 1, 0
+        time_oracle(wl, warm)
+    total_t, total_b, cores = 0.0, 0, 1
     for _ in range(args.steps):
-        dt, nb, tk, cores = time_oracle(wl, host, n_seq)
+        dt, nb, _, cores = time_oracle(wl, sample)
         total_t += dt
         total_b += nb
-        tokens += tk
     val = total_b / total_t / 1e9
-    sample = f"decode of sequences 0..{n_seq - 1} of {wl.B} per step, fp64"
+    use_shared = args.decode == "shared_prefix" or (args.decode == "auto"
+                                                    and args.config.startswith("share"))
+    cfg = config_dict(args, args.config, wl, args.step == "fused", use_shared,
+                      len(wl.cow_pairs) > 0, world)
+    sample_txt = (f"decode of sequences 0..{n_seq - 1} of {wl.B} per step "
+                  f"({sample['k_cache'].shape[0]} distinct blocks), fp64")
     return {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * total_t / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.config, "description": DESCR.get(args.config, "")},
+            "config": cfg,
             "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores,
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample_txt},
             "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
@@ -698,14 +856,21 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="mha", choices=sorted(DESCR))
+    ap.add_argument("--config", default="long", choices=sorted(DESCR),
+                    help="headline workload (default: the long-context GQA decode, the largest "
+                         "single-GPU configuration)")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload (no per_config entries)")
     ap.add_argument("--cpu-budget-rows", type=int, default=400_000_000,
                     help="query-row x token budget of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-flops", type=float, default=1.5e10,
                     help="prefill mode: causal flops of the oracle's timed sample")
-    ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
-                    help="decode step (default) or multi-query chunked-append attention")
+    ap.add_argument("--mode", choices=["decode", "prefill", "paging"], default="decode",
+                    help="decode step (default), multi-query chunked-append attention, or the "
+                         "paging-overhead control and block-size sweep")
+    ap.add_argument("--paging-configs", default="mha,gqa16,long",
+                    help="paging mode: the workloads to measure")
     ap.add_argument("--prefill-kernel", choices=["two_tile", "per_item", "single_tile"],
                     default="two_tile",
                     help="prefill kernel: warp-specialised two-tile, persistent with the "
@@ -746,8 +911,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device(f"cuda:{local_rank}"))
     try:
-        line = (run_prefill(args, rank, world, local_rank) if args.mode == "prefill"
-                else run_ours(args, rank, world, local_rank))
+        if args.mode == "prefill":
+            line = run_prefill(args, rank, world, local_rank)
+        elif args.mode == "paging":
+            line = run_paging(args, local_rank)
+        else:
+            line = run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -149,10 +149,16 @@ size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int 
  *                   use.  Each completed call leaves it ready for the next
  *                   one (its counters are back at zero).  Two calls that
  *                   share a workspace must not overlap on the GPU.  It may be
- *                   NULL when the size is 0.
+ *                   NULL when the size is 0.  After a call that raised
+ *                   PKV_DEVERR_TIMEOUT the counters may be left non-zero (the
+ *                   CTAs that stopped early took no ticket): zero-fill the
+ *                   workspace again before its next use.
  * Supported: bf16 with D in {64, 128, 256}; fp32 with D in {64, 128};
- * block_size a multiple of 16 up to 256; G = Hq / Hkv <= 16 (bf16) or <= 8
- * (fp32); num_blocks * block_size < 2^31.
+ * block_size 8, or a multiple of 16 up to 256 (the kernels stream 16-token
+ * stages; with 8-token blocks a stage is gathered from two blocks); G = Hq / Hkv
+ * <= 16 (bf16) or <= 8 (fp32); num_blocks * block_size < 2^31.  The
+ * work-balanced split (pkv_set_decode_split) needs block_size a multiple of 16;
+ * with 8-token blocks the fixed split runs.
  */
 int paged_attention_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                            const int32_t *block_tables, int max_blocks, const int32_t *seq_lens,
@@ -160,6 +166,28 @@ int paged_attention_decode(void *out, const void *q, const void *k_cache, const 
                            int64_t num_blocks, float scale, pkv_dtype dtype,
                            int partition_size, void *workspace, size_t workspace_bytes,
                            pkv_stream_t stream);
+
+/*
+ * paged_attention_decode_contiguous: the same decode over an UNPAGED cache, as a
+ * measurement control for the cost of paging.  [Index] "Limitations" says that
+ * following the block table may make a request slightly slower than a perfectly
+ * contiguous allocation; this call runs paged_attention_decode's own kernel with
+ * the block-table walk removed, so that the two can be timed on the same K/V.
+ *   k_cache, v_cache  device [B][row_stride][Hkv][D]: sequence b's token t is row
+ *                     b * row_stride + t (row_stride >= max_seq_len)
+ *   workspace         as paged_attention_decode's, sized by
+ *                     paged_attention_decode_workspace_size(B, Hq, Hkv, D,
+ *                     max_seq_len, 16, partition_size)
+ * Every other argument is paged_attention_decode's.  bf16 only (the tensor-core
+ * kernel); fixed-length partitions whatever pkv_set_decode_split says; B *
+ * row_stride < 2^31.
+ */
+int paged_attention_decode_contiguous(void *out, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *seq_lens,
+                                      int max_seq_len, int row_stride, int B, int Hq, int Hkv,
+                                      int D, float scale, pkv_dtype dtype, int partition_size,
+                                      void *workspace, size_t workspace_bytes,
+                                      pkv_stream_t stream);
 
 /*
  * paged_attention_prefill: multi-query attention over the paged cache, for
@@ -216,7 +244,11 @@ int paged_attention_prefill(void *out, const void *q, const void *k_cache, const
  * (copy-on-write of a shared block about to be written).  The other arguments,
  * the workspace rules and the supported shapes are those of
  * paged_attention_decode, with fixed-length partitions whatever
- * pkv_set_decode_split says.
+ * pkv_set_decode_split says, and the partition length (partition_size, or the
+ * library's choice) rounded up to a multiple of block_size: the block that
+ * receives a sequence's new token then lies in its last partition only.  The
+ * size from paged_attention_decode_workspace_size for the same arguments
+ * suffices (longer partitions leave fewer partials).
  */
 int paged_decode_step(void *out, const void *q, const void *k_new, const void *v_new,
                       void *k_cache, void *v_cache, const int32_t *block_tables, int max_blocks,
@@ -245,7 +277,7 @@ int paged_decode_step(void *out, const void *q, const void *k_new, const void *v
  *   prefix_lens    device [n_groups] int32: leading tokens whose blocks are
  *                  the same physical blocks in every member (equal table
  *                  entries).  The decode uses min(prefix_len, shortest member's
- *                  length - 1), rounded down to a multiple of 16.  0 means nothing shared.
+ *                  length - 1), rounded down to whole blocks.  0 means nothing shared.
  *   max_group_size host upper bound of the group sizes.
  * The other arguments are as for paged_attention_decode.  bf16 only, G <= 16.
  * The workspace (paged_attention_decode_shared_prefix_workspace_size) follows the
@@ -268,8 +300,12 @@ int paged_attention_decode_shared_prefix(void *out, const void *q, const void *k
  * does the copy-on-write copy and the new token's write, then
  * paged_attention_decode_shared_prefix, all in one launch.  The new token
  * (position seq_lens[b] - 1) must lie after the group's shared prefix; the decode
- * caps the prefix one token short of the shortest member, so that holds for any
- * prefix_lens value.  Arguments are those of the two calls.
+ * caps the prefix one token short of the shortest member and rounds it down to
+ * whole blocks, so that holds for any prefix_lens value, and the block a step
+ * rewrites is never one a prefix piece reads.  With partitions (partition_size
+ * > 0, or groups larger than 16 / G), the partition length is rounded up to a
+ * multiple of block_size, as in paged_decode_step.  Arguments are those of the
+ * two calls.
  */
 int paged_decode_step_shared_prefix(void *out, const void *q, const void *k_new,
                                     const void *v_new, void *k_cache, void *v_cache,
@@ -305,8 +341,10 @@ size_t paged_attention_decode_shared_prefix_workspace_size(int B, int Hq, int Hk
  *     PKV_NOALLOC_SCRATCH_BYTES are rejected with PKV_ERR_SCRATCH_LIMIT before
  *     anything is enqueued.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current.  Make that first call
- *     before any stream capture.
+ *     (cudaGetSymbolAddress) with that device current and keeps it for the
+ *     process.  Make that first call before any stream capture.  A
+ *     cudaDeviceReset after it is not supported: the kept address would be
+ *     stale.
  *   - All calls share the one array, and it keeps what the last call left.
  *     Each call therefore clears the part that must start at zero (the
  *     partition counters) on `stream` before the decode.  Calls that overlap
@@ -349,7 +387,10 @@ int pkv_last_cuda_error(void);
 
 /*
  * Reads the device error word of the current device into *bits, and clears it
- * when `clear` is non-zero.  This synchronises with the device.
+ * when `clear` is non-zero.  This synchronises with the device.  When
+ * PKV_DEVERR_TIMEOUT is set, the outputs of the launches that saw it are
+ * undefined, and every decode workspace they used must be zero-filled again
+ * before its next use (their partition counters may be left non-zero).
  */
 int pkv_device_errors(uint32_t *bits, int clear);
 
@@ -361,8 +402,10 @@ int pkv_device_errors(uint32_t *bits, int clear);
  * PKV_DEVERR_TIMEOUT; the device stays usable.  While that bit is set, every
  * CTA of every attention launch (decode, shared-prefix decode, prefill) returns
  * at once, whole, without reading or writing anything, so that one stall does
- * not become a wait per CTA; pkv_device_errors(&bits, 1) clears it.  Returns
- * PKV_OK or PKV_ERR_CUDA (launch failure).
+ * not become a wait per CTA; pkv_device_errors(&bits, 1) clears it.  Such a
+ * CTA takes no partition ticket, so a workspace used while the bit was set must
+ * be zero-filled again before its next use.  Returns PKV_OK or PKV_ERR_CUDA
+ * (launch failure).
  */
 int pkv_debug_stalled_wait(pkv_stream_t stream);
 

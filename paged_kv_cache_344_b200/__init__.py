@@ -80,6 +80,9 @@ def lib() -> ctypes.CDLL:
     L.paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
                                          i32, i64, f32, i32, i32, vp, sz, vp]
     L.paged_attention_decode.restype = i32
+    L.paged_attention_decode_contiguous.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                                    i32, f32, i32, i32, vp, sz, vp]
+    L.paged_attention_decode_contiguous.restype = i32
     L.paged_attention_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
     L.paged_attention_prefill_workspace_size.restype = sz
     L.paged_attention_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
@@ -189,6 +192,19 @@ def paged_attention_decode(out, q, k_cache, v_cache, block_tables, seq_lens, max
         block_tables.shape[1], _ptr(seq_lens), int(max_seq_len), B, Hq, Hkv, D, bs, NB,
         float(scale), _dtype_code(q), int(partition_size), _ptr(workspace), ws_bytes,
         _stream(q, stream)))
+
+
+def paged_attention_decode_contiguous(out, q, k_cache, v_cache, seq_lens, max_seq_len, scale,
+                                      workspace=None, partition_size=0, stream=None) -> None:
+    """The decode over an unpaged cache ``k_cache, v_cache [B, row_stride, Hkv, D]`` (the
+    paging-overhead control: the same kernel without the block-table walk)."""
+    B, Hq, D = q.shape
+    stride, Hkv = k_cache.shape[1], k_cache.shape[2]
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("paged_attention_decode_contiguous", lib().paged_attention_decode_contiguous(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(max_seq_len),
+        stride, B, Hq, Hkv, D, float(scale), _dtype_code(q), int(partition_size),
+        _ptr(workspace), ws_bytes, _stream(q, stream)))
 
 
 def paged_attention_prefill_workspace_size(B, Hq, Hkv, max_q_len) -> int:

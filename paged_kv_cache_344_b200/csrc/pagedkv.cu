@@ -24,7 +24,13 @@ std::atomic<int> g_decode_ctas{0};  // 0: as many as fit (at most 2 per SM)
 std::atomic<int> g_decode_split{PKV_SPLIT_FIXED};
 std::atomic<int> g_prefill_path{PKV_PREFILL_AUTO};
 
-constexpr int kSmCount = 148;  // B200
+// SM count the partition choice is tuned for (B200).  It is a constant, not
+// the device's attribute, so that the partition length and the workspace size
+// stay pure functions of the arguments (no CUDA call, no device state): the
+// caller can size a workspace before choosing a device or stream.  On a
+// device with another SM count the choice stays correct, only its wave count
+// is tuned for 148 SMs.
+constexpr int kSmCount = 148;
 
 // Multiprocessors of the current device (looked up once per device).
 cudaError_t sm_count(int* out) {
@@ -70,13 +76,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 int make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t rows,
-                   pkv_dtype dtype, bool swizzle) {
+                   pkv_dtype dtype, bool swizzle, int box_rows = pkv::kStageTokens) {
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   const int es = dtype == PKV_BF16 ? 2 : 4;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)D * es, (cuuint64_t)Hkv * D * es};
-  cuuint32_t box[3] = {(cuuint32_t)(swizzle ? 64 : D), 1u, (cuuint32_t)pkv::kStageTokens};
+  cuuint32_t box[3] = {(cuuint32_t)(swizzle ? 64 : D), 1u, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(map, dtype == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
@@ -95,14 +101,16 @@ int make_cache_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t r
 // tokens, 64-dim halves, KV heads) with a box of {64, 16, D / 64, 1}, so that
 // one TMA load brings a 16-token tile as D / 64 swizzled 16 x 128 B sub-tiles.
 // The dims of one token are contiguous, so its halves lie 128 bytes apart.
+// `half_box` (8-token blocks): a box of {64, 8, 1, 1}, one half of one sub-tile.
 int make_stage_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t rows,
-                   pkv_dtype dtype) {
+                   pkv_dtype dtype, bool half_box = false) {
   if (dtype != PKV_BF16 || D % 64 != 0) return PKV_ERR_UNSUPPORTED;
   auto fn = encode_fn();
   if (!fn) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[4] = {64u, (cuuint64_t)rows, (cuuint64_t)(D / 64), (cuuint64_t)Hkv};
   cuuint64_t strides[3] = {(cuuint64_t)Hkv * D * 2, 128u, (cuuint64_t)D * 2};
-  cuuint32_t box[4] = {64u, (cuuint32_t)pkv::kStageTokens, (cuuint32_t)(D / 64), 1u};
+  cuuint32_t box[4] = {64u, (cuuint32_t)(half_box ? pkv::kStageTokens / 2 : pkv::kStageTokens),
+                       (cuuint32_t)(half_box ? 1 : D / 64), 1u};
   cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -155,8 +163,14 @@ struct DecodeShape {
   size_t ws_bytes;                // size reported to callers: covers either split
 };
 
+// `fused` (paged_decode_step): fixed-length partitions whatever the split mode,
+// and a partition length rounded up to whole blocks.  The step rewrites the
+// block that receives each sequence's new token (copy-on-write copy and the new
+// row) from the CTA of the sequence's last partition, so no other partition may
+// hold tokens of that block.  `fixed_only`: fixed-length partitions, nothing else.
 int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
-                 int partition_size, DecodeShape* s, bool force_fixed = false) {
+                 int partition_size, DecodeShape* s, bool fused = false,
+                 bool fixed_only = false) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || max_seq_len < 0)
     return PKV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
@@ -166,7 +180,8 @@ int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
   auto align256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
 
   // Fixed-length partitions (the default split).
-  const int P = partition_size > 0 ? partition_size : auto_partition(B, Hkv, max_seq_len);
+  int P = partition_size > 0 ? partition_size : auto_partition(B, Hkv, max_seq_len);
+  if (fused && P % block_size != 0) P = (int)ceil_div(P, block_size) * block_size;
   const int64_t mp = max_seq_len > 0 ? ceil_div(max_seq_len, P) : 1;
   if (mp > 65535) return PKV_ERR_OUT_OF_RANGE;
   size_t f_ml = 0, f_acc = 0, f_bytes = 0;
@@ -178,7 +193,8 @@ int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
   // Work-balanced split (opt-in): needs the per-sequence prefix in shared memory
   // and a stage count that fits in 31 bits.
   const int64_t max_stages = (int64_t)B * Hkv * ceil_div(max_seq_len, pkv::kStageTokens);
-  const bool bal_ok = partition_size == 0 && B <= pkv::kBalancedMaxB && max_stages < 0x7fffffffLL;
+  const bool bal_ok = partition_size == 0 && B <= pkv::kBalancedMaxB && max_stages < 0x7fffffffLL &&
+                      block_size % pkv::kStageTokens == 0;
   size_t b_ml = 0, b_acc = 0, b_bytes = 0;
   if (bal_ok && B > 0) {
     const size_t slots = pkv::balanced_slots((size_t)B, (size_t)Hkv);
@@ -186,7 +202,7 @@ int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
     b_acc = b_ml + align256(slots * G * sizeof(float2));
     b_bytes = b_acc + slots * G * (size_t)D * sizeof(float);
   }
-  s->balanced = bal_ok && !force_fixed &&
+  s->balanced = bal_ok && !fused && !fixed_only &&
                 g_decode_split.load(std::memory_order_relaxed) == PKV_SPLIT_BALANCED;
   s->P = s->balanced ? 0 : P;
   s->max_parts = s->balanced ? 0 : (int)mp;
@@ -197,10 +213,10 @@ int decode_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
   return PKV_OK;
 }
 
-template <class C, typename T, int D>
+template <class C, typename T, int D, int LAYOUT>
 int launch_decode(const pkv::DecodeParams& p, int B, const CUtensorMap& mk, const CUtensorMap& mv,
                   cudaStream_t stream) {
-  auto kernel = pkv::paged_decode_kernel<C, T, D>;
+  auto kernel = pkv::paged_decode_kernel<C, T, D, LAYOUT>;
   const size_t smem = pkv::DecodeSmem<C>::kBytes;
   static std::atomic<uint64_t> smem_set{0};
   int rc = ensure_smem(kernel, smem, smem_set);
@@ -242,27 +258,33 @@ int launch_balanced(const pkv::DecodeParams& p, const CUtensorMap& mk, const CUt
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
-template <class C, typename T, int D>
+// The balanced split exists for the plain block layout only (decode_shape never
+// picks it for another layout).
+template <class C, typename T, int D, int LAYOUT>
 int launch_any(const pkv::DecodeParams& p, bool balanced, const CUtensorMap& mk,
                const CUtensorMap& mv, cudaStream_t s) {
-  return balanced ? launch_balanced<C, T, D>(p, mk, mv, s) : launch_decode<C, T, D>(p, p.B, mk, mv, s);
+  if constexpr (LAYOUT == pkv::kLayoutPaged) {
+    if (balanced) return launch_balanced<C, T, D>(p, mk, mv, s);
+  }
+  return launch_decode<C, T, D, LAYOUT>(p, p.B, mk, mv, s);
 }
 
-template <typename T, int D>
+template <typename T, int D, int LAYOUT>
 int dispatch_simt(const pkv::DecodeParams& p, bool bal, const CUtensorMap& mk,
                   const CUtensorMap& mv, cudaStream_t s) {
-  if (p.G == 1) return launch_any<pkv::SimtConsumer<T, D, 1>, T, D>(p, bal, mk, mv, s);
-  if (p.G == 2) return launch_any<pkv::SimtConsumer<T, D, 2>, T, D>(p, bal, mk, mv, s);
-  if (p.G <= 4) return launch_any<pkv::SimtConsumer<T, D, 4>, T, D>(p, bal, mk, mv, s);
-  if (p.G <= 8) return launch_any<pkv::SimtConsumer<T, D, 8>, T, D>(p, bal, mk, mv, s);
+  if (p.G == 1) return launch_any<pkv::SimtConsumer<T, D, 1>, T, D, LAYOUT>(p, bal, mk, mv, s);
+  if (p.G == 2) return launch_any<pkv::SimtConsumer<T, D, 2>, T, D, LAYOUT>(p, bal, mk, mv, s);
+  if (p.G <= 4) return launch_any<pkv::SimtConsumer<T, D, 4>, T, D, LAYOUT>(p, bal, mk, mv, s);
+  if (p.G <= 8) return launch_any<pkv::SimtConsumer<T, D, 8>, T, D, LAYOUT>(p, bal, mk, mv, s);
   return PKV_ERR_UNSUPPORTED;
 }
 
-template <int D>
+template <int D, int LAYOUT>
 int dispatch_mma(const pkv::DecodeParams& p, bool bal, const CUtensorMap& mk,
                  const CUtensorMap& mv, cudaStream_t s) {
-  if (p.G <= 8) return launch_any<pkv::MmaConsumer<D, 1>, __nv_bfloat16, D>(p, bal, mk, mv, s);
-  if (p.G <= 16) return launch_any<pkv::MmaConsumer<D, 2>, __nv_bfloat16, D>(p, bal, mk, mv, s);
+  using T = __nv_bfloat16;
+  if (p.G <= 8) return launch_any<pkv::MmaConsumer<D, 1>, T, D, LAYOUT>(p, bal, mk, mv, s);
+  if (p.G <= 16) return launch_any<pkv::MmaConsumer<D, 2>, T, D, LAYOUT>(p, bal, mk, mv, s);
   return PKV_ERR_UNSUPPORTED;
 }
 
@@ -283,8 +305,11 @@ struct SharedShape {
   size_t off_ml, off_acc, bytes;
 };
 
+// `fused` (paged_decode_step_shared_prefix): the partition length is rounded up to
+// whole blocks, so that the block receiving a sequence's new token lies in its
+// last own partition only (see decode_shape).
 int shared_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
-                 int partition_size, SharedShape* s) {
+                 int partition_size, SharedShape* s, bool fused = false) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || block_size <= 0 || max_seq_len < 0)
     return PKV_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return PKV_ERR_INVALID_ARG;
@@ -293,6 +318,7 @@ int shared_shape(int B, int Hq, int Hkv, int D, int max_seq_len, int block_size,
   // query rows; long partitions keep their count (and the partials) low.
   // Measured on B200 (shared-prefix workloads): 2048 beats 1024 and 512.
   s->P = partition_size > 0 ? partition_size : std::max(2048, auto_partition(B, Hkv, max_seq_len));
+  if (fused && s->P % block_size != 0) s->P = (int)ceil_div(s->P, block_size) * block_size;
   const int64_t mp = std::max<int64_t>(1, ceil_div(max_seq_len, s->P));
   if (mp > 32767) return PKV_ERR_OUT_OF_RANGE;
   s->max_pp = (int)mp;
@@ -400,12 +426,35 @@ size_t paged_attention_decode_workspace_size(int B, int Hq, int Hkv, int D, int 
 
 namespace {
 
-// The fused step's extra inputs (all null for a plain decode).
+// The fused step's extra inputs (all null for a plain decode), and the flag of
+// the unpaged control (paged_attention_decode_contiguous).
 struct StepArgs {
   const void* k_new = nullptr;
   const void* v_new = nullptr;
   const int32_t* cow_src = nullptr;
+  bool contiguous = false;
 };
+
+template <int LAYOUT>
+int dispatch_layout(const pkv::DecodeParams& p, bool tc, bool bal, pkv_dtype dtype, int D,
+                    const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
+  if (tc) {
+    if (D == 64) return dispatch_mma<64, LAYOUT>(p, bal, mk, mv, stream);
+    if (D == 128) return dispatch_mma<128, LAYOUT>(p, bal, mk, mv, stream);
+    return dispatch_mma<256, LAYOUT>(p, bal, mk, mv, stream);
+  }
+  if constexpr (LAYOUT == pkv::kLayoutContig) {
+    return PKV_ERR_UNSUPPORTED;  // the unpaged control runs the tensor-core kernels only
+  } else {
+    if (dtype == PKV_BF16) {
+      if (D == 64) return dispatch_simt<__nv_bfloat16, 64, LAYOUT>(p, bal, mk, mv, stream);
+      if (D == 128) return dispatch_simt<__nv_bfloat16, 128, LAYOUT>(p, bal, mk, mv, stream);
+      return dispatch_simt<__nv_bfloat16, 256, LAYOUT>(p, bal, mk, mv, stream);
+    }
+    if (D == 64) return dispatch_simt<float, 64, LAYOUT>(p, bal, mk, mv, stream);
+    return dispatch_simt<float, 128, LAYOUT>(p, bal, mk, mv, stream);
+  }
+}
 
 int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cache,
                 const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
@@ -414,14 +463,17 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 void* workspace, size_t workspace_bytes, pkv_stream_t stream,
                 const StepArgs& step) {
   const bool fused = step.k_new != nullptr;
+  const bool contig = step.contiguous;
   if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
   DecodeShape shape;
-  int rc = decode_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape, fused);
+  int rc = decode_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape, fused,
+                        contig);
   if (rc != PKV_OK) return rc;
   if (max_blocks <= 0 || num_blocks <= 0 || !std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
   if (B == 0) return PKV_OK;
   if (B > 65535) return PKV_ERR_OUT_OF_RANGE;
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens) return PKV_ERR_INVALID_ARG;
+  if (!out || !q || !k_cache || !v_cache || (!block_tables && !contig) || !seq_lens)
+    return PKV_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
       (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
@@ -429,7 +481,10 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   const int G = Hq / Hkv;
   const bool d_ok = dtype == PKV_BF16 ? (D == 64 || D == 128 || D == 256) : (D == 64 || D == 128);
   if (!d_ok) return PKV_ERR_UNSUPPORTED;
-  if (block_size % pkv::kStageTokens != 0 || block_size > 256) return PKV_ERR_UNSUPPORTED;
+  // Blocks of 8 tokens (a 16-token stage from two blocks) or multiples of 16.
+  const bool bs8 = !contig && block_size == pkv::kStageTokens / 2;
+  if (!contig && !bs8 && (block_size % pkv::kStageTokens != 0 || block_size > 256))
+    return PKV_ERR_UNSUPPORTED;
   if (G > (dtype == PKV_BF16 ? 16 : 8)) return PKV_ERR_UNSUPPORTED;
   if (num_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
   if ((int64_t)max_blocks > 0x7fffffffLL / block_size) return PKV_ERR_OUT_OF_RANGE;
@@ -471,28 +526,21 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   }
 
   const bool tc = use_tensor_cores(dtype, G);
+  if (contig && !tc) return PKV_ERR_UNSUPPORTED;
   CUtensorMap mk, mv;
   const int64_t rows = num_blocks * block_size;
-  if ((rc = tc ? make_stage_map(&mk, k_cache, D, Hkv, rows, dtype)
-                : make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, false)) != PKV_OK)
+  const int box_rows = bs8 ? pkv::kStageTokens / 2 : pkv::kStageTokens;
+  if ((rc = tc ? make_stage_map(&mk, k_cache, D, Hkv, rows, dtype, bs8)
+                : make_cache_map(&mk, k_cache, D, Hkv, rows, dtype, false, box_rows)) != PKV_OK)
     return rc;
-  if ((rc = tc ? make_stage_map(&mv, v_cache, D, Hkv, rows, dtype)
-                : make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, false)) != PKV_OK)
+  if ((rc = tc ? make_stage_map(&mv, v_cache, D, Hkv, rows, dtype, bs8)
+                : make_cache_map(&mv, v_cache, D, Hkv, rows, dtype, false, box_rows)) != PKV_OK)
     return rc;
 
   const bool bal = shape.balanced;
-  if (tc) {
-    if (D == 64) return dispatch_mma<64>(p, bal, mk, mv, stream);
-    if (D == 128) return dispatch_mma<128>(p, bal, mk, mv, stream);
-    return dispatch_mma<256>(p, bal, mk, mv, stream);
-  }
-  if (dtype == PKV_BF16) {
-    if (D == 64) return dispatch_simt<__nv_bfloat16, 64>(p, bal, mk, mv, stream);
-    if (D == 128) return dispatch_simt<__nv_bfloat16, 128>(p, bal, mk, mv, stream);
-    return dispatch_simt<__nv_bfloat16, 256>(p, bal, mk, mv, stream);
-  }
-  if (D == 64) return dispatch_simt<float, 64>(p, bal, mk, mv, stream);
-  return dispatch_simt<float, 128>(p, bal, mk, mv, stream);
+  if (contig) return dispatch_layout<pkv::kLayoutContig>(p, tc, false, dtype, D, mk, mv, stream);
+  if (bs8) return dispatch_layout<pkv::kLayoutPaged8>(p, tc, false, dtype, D, mk, mv, stream);
+  return dispatch_layout<pkv::kLayoutPaged>(p, tc, bal, dtype, D, mk, mv, stream);
 }
 
 }  // namespace
@@ -507,6 +555,22 @@ int paged_attention_decode(void* out, const void* q, const void* k_cache, const 
   return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks, seq_lens, max_seq_len, B,
                      Hq, Hkv, D, block_size, num_blocks, scale, dtype, partition_size, workspace,
                      workspace_bytes, stream, StepArgs{});
+}
+
+int paged_attention_decode_contiguous(void* out, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* seq_lens,
+                                      int max_seq_len, int row_stride, int B, int Hq, int Hkv,
+                                      int D, float scale, pkv_dtype dtype, int partition_size,
+                                      void* workspace, size_t workspace_bytes,
+                                      pkv_stream_t stream) {
+  if (row_stride <= 0 || row_stride < max_seq_len) return PKV_ERR_INVALID_ARG;
+  if (dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  StepArgs contig;
+  contig.contiguous = true;
+  // Sequence b is "block" b of row_stride tokens, and the kernel never reads a table.
+  return decode_impl(out, q, k_cache, v_cache, nullptr, 1, seq_lens, max_seq_len, B, Hq, Hkv, D,
+                     row_stride, std::max(B, 1), scale, dtype, partition_size, workspace,
+                     workspace_bytes, stream, contig);
 }
 
 int paged_decode_step(void* out, const void* q, const void* k_new, const void* v_new,
@@ -546,7 +610,8 @@ int shared_impl(void* out, const void* q, const void* k_cache, const void* v_cac
                 const StepArgs& step) {
   if (dtype != PKV_BF16 && dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
   SharedShape shape;
-  int rc = shared_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape);
+  int rc = shared_shape(B, Hq, Hkv, D, max_seq_len, block_size, partition_size, &shape,
+                        step.k_new != nullptr);
   if (rc != PKV_OK) return rc;
   if (max_blocks <= 0 || num_blocks <= 0 || !std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
   if (n_groups <= 0 || max_group_size <= 0) return PKV_ERR_INVALID_ARG;

@@ -32,6 +32,15 @@
 namespace pkv {
 
 constexpr int kStageTokens = 16;  // tokens per TMA box / pipeline stage
+
+// Stages a warp prefetches into L2 ahead of its ring (tensor-core consumers).  A
+// warp keeps only kStages stages in flight into shared memory; the L2 prefetches
+// of the next ones put more bytes in flight without holding shared memory, so the
+// ring's own loads hit L2.
+#ifndef PKV_PREFETCH_STAGES
+#define PKV_PREFETCH_STAGES 0
+#endif
+constexpr int kPrefetchStages = PKV_PREFETCH_STAGES;
 constexpr int kWarps = 4;         // consumer warps per CTA
 constexpr uint32_t kFull = 0xffffffffu;
 
@@ -148,6 +157,9 @@ struct SimtConsumer {
   static constexpr int kStages = ROWB <= 128 ? 6 : (ROWB <= 256 ? 3 : 2);
   static constexpr int GP = GMAX;
   static constexpr bool kSwizzle = false;
+  static constexpr bool kCanPrefetch = false;  // (3-D maps; no L2 prefetch path)
+  static __device__ __forceinline__ void prefetch_stage(const CUtensorMap*, const CUtensorMap*,
+                                                        int, int) {}
   static_assert(LPT >= 1 && LPT <= 32 && TPI * LPT == 32, "bad lane split");
 
   float qv[GMAX][2][EPC];
@@ -185,7 +197,28 @@ struct SimtConsumer {
     tma_load_3d(st + kTileBytes, tv, bar, 0, kvh, row, pol);
   }
 
-  __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane) {
+  // Blocks of 8 tokens: the stage's two halves come from two blocks (8-row boxes).
+  static __device__ __forceinline__ void load_stage_halves(uint8_t* st, const CUtensorMap* tk,
+                                                           const CUtensorMap* tv, uint64_t* bar,
+                                                           int kvh, int row0, int row1,
+                                                           uint64_t pol) {
+    constexpr int kHalf = kStageTokens / 2 * ROWB;
+    tma_load_3d(st, tk, bar, 0, kvh, row0, pol);
+    tma_load_3d(st + kHalf, tk, bar, 0, kvh, row1, pol);
+    tma_load_3d(st + kTileBytes, tv, bar, 0, kvh, row0, pol);
+    tma_load_3d(st + kTileBytes + kHalf, tv, bar, 0, kvh, row1, pol);
+  }
+
+  // `release()` (warp-collective) is called once the stage's shared memory is no
+  // longer needed; here that is after the whole stage.
+  template <class Release>
+  __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane, Release&& release) {
+    consume_body(st, n_valid, lane);
+    __syncwarp();
+    release();
+  }
+
+  __device__ __forceinline__ void consume_body(uint8_t* st, int n_valid, int lane) {
     const uint8_t* sk = st;
     const uint8_t* sv = st + kTileBytes;
     const int sub = lane % LPT;
@@ -311,6 +344,10 @@ struct MmaConsumer {
   static constexpr int MT = D / 16;
   static constexpr int GP = 8 * NT;
   static constexpr bool kSwizzle = true;
+  static constexpr bool kCanPrefetch = true;
+  // V fragments held in registers so that the stage is released before the
+  // softmax (D <= 128; at D = 256 they would not fit next to O).
+  static constexpr bool kEarly = D <= 128;
 
   uint32_t qf[NT][KS][2];
   float m[NT][2], l[NT][2];
@@ -383,25 +420,59 @@ struct MmaConsumer {
     tma_load_4d(st + kTileBytes, tv, bar, 0, row, 0, kvh, pol);
   }
 
+  // An L2 prefetch of the stage's K and V boxes (a later load_stage finds them there).
+  static __device__ __forceinline__ void prefetch_stage(const CUtensorMap* tk,
+                                                        const CUtensorMap* tv, int kvh, int row) {
+    tma_prefetch_4d(tk, 0, row, 0, kvh);
+    tma_prefetch_4d(tv, 0, row, 0, kvh);
+  }
+
+  // Blocks of 8 tokens: the maps' box is {64, 8, 1, 1}, and each 64-dim sub-tile is
+  // filled by two boxes, rows 0..7 from the first block and 8..15 from the second.
+  // The second box lands 1024 bytes in, where the 128-byte swizzle pattern repeats,
+  // so the sub-tile reads exactly like one 16-row box.
+  static __device__ __forceinline__ void load_stage_halves(uint8_t* st, const CUtensorMap* tk,
+                                                           const CUtensorMap* tv, uint64_t* bar,
+                                                           int kvh, int row0, int row1,
+                                                           uint64_t pol) {
+#pragma unroll
+    for (int sb = 0; sb < SUB; ++sb) {
+      uint8_t* k = st + sb * kSubBytes;
+      uint8_t* v = k + kTileBytes;
+      tma_load_4d(k, tk, bar, 0, row0, sb, kvh, pol);
+      tma_load_4d(k + kSubBytes / 2, tk, bar, 0, row1, sb, kvh, pol);
+      tma_load_4d(v, tv, bar, 0, row0, sb, kvh, pol);
+      tma_load_4d(v + kSubBytes / 2, tv, bar, 0, row1, sb, kvh, pol);
+    }
+  }
+
   // Byte offset of (row, 16-byte chunk) inside a swizzled 16x128 B sub-tile.
   static __device__ __forceinline__ uint32_t swz(int row, int chunk) {
     return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
   }
 
-  __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane) {
-    consume_impl<false>(st, n_valid, lane, 0, GP);
+  // Consumes one stage; `release()` (warp-collective) is called as soon as the
+  // stage's shared memory has been read (K by the score MMAs, V into registers),
+  // so that the warp can refill the slot while it still computes the softmax and
+  // the P V product.
+  template <class Release>
+  __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane, Release&& release) {
+    consume_impl<false>(st, n_valid, lane, 0, GP, release);
   }
 
   // The same, with only query rows [r0, r1) of the N dimension scoring this
   // stage (the others see it as masked): a stage of one member's own tokens in a
   // shared-prefix group.  A row may then have seen no token yet, so the
   // rescale factors are guarded against -inf - -inf.
-  __device__ __forceinline__ void consume_rows(uint8_t* st, int n_valid, int lane, int r0, int r1) {
-    consume_impl<true>(st, n_valid, lane, r0, r1);
+  template <class Release>
+  __device__ __forceinline__ void consume_rows(uint8_t* st, int n_valid, int lane, int r0, int r1,
+                                               Release&& release) {
+    consume_impl<true>(st, n_valid, lane, r0, r1, release);
   }
 
-  template <bool kRows>
-  __device__ __forceinline__ void consume_impl(uint8_t* st, int n_valid, int lane, int r0, int r1) {
+  template <bool kRows, class Release>
+  __device__ __forceinline__ void consume_impl(uint8_t* st, int n_valid, int lane, int r0, int r1,
+                                               Release& release) {
     const uint32_t sk = smem_u32(st);
     const uint32_t sv = sk + kTileBytes;
     const int mi = lane / 8, rr = lane % 8;
@@ -431,10 +502,43 @@ struct MmaConsumer {
 #pragma unroll
       for (int j = 0; j < 4; ++j) s[nt][j] += s2[nt][j];
 
-    // Invalid tail slots of the last stage hold anything (even NaN): their
-    // scores are replaced by -inf, and their V rows are zeroed before the PV
-    // product so that 0 * NaN cannot reach the accumulator.
-    if (n_valid < kStageTokens) {
+    // V^T fragments (A operand of O^T += V^T P): lane (g, t) = (lane / 4, lane % 4)
+    // holds dims (g, g + 8) of each 16-dim tile for tokens (2t, 2t + 1) in
+    // va[mt][0..1] and (2t + 8, 2t + 9) in va[mt][2..3].  Up to D = 128 they are
+    // read into registers here and the slot is released at once; at D = 256 the
+    // registers do not suffice, V is read during the P V product and the slot is
+    // released after it.
+    uint32_t va[kEarly ? MT : 1][4];
+    auto load_v = [&](int mt, uint32_t (&a)[4]) {
+      const int t = (mi >> 1) * 8 + rr;
+      const int d0 = mt * 16 + (mi & 1) * 8;
+      ldmatrix_x4_trans(sv + (d0 / 64) * kSubBytes + swz(t, (d0 % 64) / 8), a[0], a[1], a[2], a[3]);
+    };
+    if constexpr (kEarly) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) load_v(mt, va[mt]);
+      // Invalid tail slots of the last stage hold anything (even NaN): their V
+      // values are zeroed here, in registers, so that 0 * NaN cannot reach the
+      // accumulator (their scores become -inf below).
+      if (n_valid < kStageTokens) {
+        const int t2 = 2 * (lane % 4);
+        const uint32_t lo = (t2 < n_valid ? 0x0000ffffu : 0u) | (t2 + 1 < n_valid ? 0xffff0000u : 0u);
+        const uint32_t hi = (t2 + 8 < n_valid ? 0x0000ffffu : 0u) | (t2 + 9 < n_valid ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          va[mt][0] &= lo;
+          va[mt][1] &= lo;
+          va[mt][2] &= hi;
+          va[mt][3] &= hi;
+        }
+      }
+      // Every read of the stage is issued; order them before the refill (an
+      // async-proxy write into the same slot) and hand the slot back.
+      fence_proxy_async_smem();
+      __syncwarp();
+      release();
+    } else if (n_valid < kStageTokens) {
+      // The same masking in shared memory: the invalid V rows become zeros.
       uint4* vz = reinterpret_cast<uint4*>(st + kTileBytes);
       const int nvec = (kStageTokens - n_valid) * 8;  // 128-byte rows, per sub-tile
 #pragma unroll
@@ -471,40 +575,36 @@ struct MmaConsumer {
         mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
       }
       const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
-      float al0 = exp2f(m[nt][0] - mn0), al1 = exp2f(m[nt][1] - mn1);
-      if (kRows) {  // a row with no token so far keeps m = -inf and l = o = 0
-        al0 = mn0 == -INFINITY ? 1.f : al0;
-        al1 = mn1 == -INFINITY ? 1.f : al1;
-      }
-      m[nt][0] = mn0;
-      m[nt][1] = mn1;
-      if (kRows) {
-        const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
-        x[0] = exp2f(x[0] - b0);
-        x[1] = exp2f(x[1] - b1);
-        x[2] = exp2f(x[2] - b0);
-        x[3] = exp2f(x[3] - b1);
-      } else {
-        x[0] = exp2f(x[0] - mn0);
-        x[1] = exp2f(x[1] - mn1);
-        x[2] = exp2f(x[2] - mn0);
-        x[3] = exp2f(x[3] - mn1);
-      }
-      float sum0 = x[0] + x[2], sum1 = x[1] + x[3];
+      // O and l are rescaled only when some row's maximum moved (one vote);
+      // otherwise every factor is exactly 1.
+      if (__any_sync(kFull, (mn0 != m[nt][0]) || (mn1 != m[nt][1]))) {
+        float al0 = ex2_approx(m[nt][0] - mn0), al1 = ex2_approx(m[nt][1] - mn1);
+        if (kRows) {  // a row with no token so far keeps m = -inf and l = o = 0
+          al0 = mn0 == -INFINITY ? 1.f : al0;
+          al1 = mn1 == -INFINITY ? 1.f : al1;
+        }
+        l[nt][0] *= al0;
+        l[nt][1] *= al1;
 #pragma unroll
-      for (int off = 4; off < 32; off *= 2) {
-        sum0 += __shfl_xor_sync(kFull, sum0, off);
-        sum1 += __shfl_xor_sync(kFull, sum1, off);
+        for (int mt = 0; mt < MT; ++mt) {
+          o[nt][mt][0] *= al0;
+          o[nt][mt][1] *= al1;
+          o[nt][mt][2] *= al0;
+          o[nt][mt][3] *= al1;
+        }
+        m[nt][0] = mn0;
+        m[nt][1] = mn1;
       }
-      l[nt][0] = l[nt][0] * al0 + sum0;
-      l[nt][1] = l[nt][1] * al1 + sum1;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        o[nt][mt][0] *= al0;
-        o[nt][mt][1] *= al1;
-        o[nt][mt][2] *= al0;
-        o[nt][mt][3] *= al1;
-      }
+      const float b0 = kRows && mn0 == -INFINITY ? 0.f : mn0;
+      const float b1 = kRows && mn1 == -INFINITY ? 0.f : mn1;
+      x[0] = ex2_approx(x[0] - b0);
+      x[1] = ex2_approx(x[1] - b1);
+      x[2] = ex2_approx(x[2] - b0);
+      x[3] = ex2_approx(x[3] - b1);
+      // Row sums stay per lane (each lane's share of its column); they are added
+      // across the column's eight lanes only when the state is read out.
+      l[nt][0] += x[0] + x[2];
+      l[nt][1] += x[1] + x[3];
       // P (rows t, cols g) -> B fragment of P with k = t, n = g.
       pb[nt][0] = movmatrix_trans(pack_bf16x2(x[0], x[1]));
       pb[nt][1] = movmatrix_trans(pack_bf16x2(x[2], x[3]));
@@ -513,26 +613,36 @@ struct MmaConsumer {
     // O^T += V^T P: one m16n8k16 per (16-dim tile, head tile).
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      const int t = (mi >> 1) * 8 + rr;
-      const int d0 = mt * 16 + (mi & 1) * 8;
-      uint32_t a[4];
-      ldmatrix_x4_trans(sv + (d0 / 64) * kSubBytes + swz(t, (d0 % 64) / 8), a[0], a[1], a[2],
-                        a[3]);
+      if constexpr (!kEarly) load_v(mt, va[0]);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
-        if (live(nt)) mma_bf16_16816(o[nt][mt], a, pb[nt][0], pb[nt][1]);
+        if (live(nt)) mma_bf16_16816(o[nt][mt], va[kEarly ? mt : 0], pb[nt][0], pb[nt][1]);
     }
+    if constexpr (!kEarly) {
+      __syncwarp();
+      release();
+    }
+  }
+
+  // Row sum of column pair (2 (lane % 4), +1) of head tile nt: the per-lane
+  // shares added over the eight lanes that hold the column.
+  __device__ __forceinline__ float row_sum(int nt, int j) const {
+    float x = l[nt][j];
+#pragma unroll
+    for (int off = 4; off < 32; off *= 2) x += __shfl_xor_sync(kFull, x, off);
+    return x;
   }
 
   __device__ __forceinline__ void store_state(float* dst, int lane) const {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int g = nt * 8 + 2 * (lane % 4);
+      const float l0 = row_sum(nt, 0), l1 = row_sum(nt, 1);
       if (lane < 4) {
         dst[g] = m[nt][0];
         dst[g + 1] = m[nt][1];
-        dst[GP + g] = l[nt][0];
-        dst[GP + g + 1] = l[nt][1];
+        dst[GP + g] = l0;
+        dst[GP + g + 1] = l1;
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -550,7 +660,7 @@ struct MmaConsumer {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int g = nt * 8 + 2 * (lane % 4);
-      const float i0 = 1.f / l[nt][0], i1 = 1.f / l[nt][1];
+      const float i0 = 1.f / row_sum(nt, 0), i1 = 1.f / row_sum(nt, 1);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         const int d = mt * 16 + lane / 4;
@@ -571,9 +681,10 @@ struct MmaConsumer {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int g = nt * 8 + 2 * (lane % 4);
+      const float l0 = row_sum(nt, 0), l1 = row_sum(nt, 1);
       if (lane < 4) {
-        if (g < G) ml_dst[g] = make_float2(m[nt][0], l[nt][0]);
-        if (g + 1 < G) ml_dst[g + 1] = make_float2(m[nt][1], l[nt][1]);
+        if (g < G) ml_dst[g] = make_float2(m[nt][0], l0);
+        if (g + 1 < G) ml_dst[g + 1] = make_float2(m[nt][1], l1);
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -646,7 +757,15 @@ struct DecodeSmem {
       1024 /*alignment slack*/ + (size_t)kWarps * kRingBytes + kWarps * C::kStages * 8;
 };
 
-template <class C, typename T, int D>
+// Where a stage's K/V rows are found.
+enum : int {
+  kLayoutPaged = 0,   // block_size a multiple of 16: a 16-token stage lies in one block
+  kLayoutPaged8 = 1,  // block_size 8: a stage spans two blocks (two 8-token boxes)
+  kLayoutContig = 2,  // unpaged cache [B][bs][Hkv][D] (bs = the row stride of a sequence):
+                      // no block table at all; the control for the paging overhead
+};
+
+template <class C, typename T, int D, int LAYOUT = kLayoutPaged>
 __global__ void __launch_bounds__(kWarps * 32)
     paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV) {
@@ -703,41 +822,82 @@ __global__ void __launch_bounds__(kWarps * 32)
 
   const uint64_t pol = l2_policy_evict_first();
   const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks;
-  auto stage_id = [&](int k) -> int {
-    const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
+  // Physical id of the block holding tokens t0 + 8 * half .. of stage k (half 1 only
+  // with 8-token blocks, and only when the partition has tokens there).
+  auto stage_id = [&](int k, int half) -> int {
+    const int t0 = t_begin + (warp + kWarps * k) * kStageTokens + 8 * half;
+    if constexpr (LAYOUT == kLayoutContig) return b;
+    if (half && t0 >= t_end) return 0;
     return bt_row[t0 / p.bs];
   };
-  // Physical ids of this warp's stages win_base .. win_base+63 (one per lane, two windows).
+  // Physical ids of this warp's stages win_base .. win_base+63 (one per lane, two
+  // windows; with 8-token blocks a second pair for the stages' second halves).
+  constexpr bool kTwo = LAYOUT == kLayoutPaged8;
+  constexpr int kPrefetch = C::kCanPrefetch && !kTwo ? kPrefetchStages : 0;
   int win_base = 0;
-  int win0 = lane < n_w ? stage_id(lane) : -1;
-  int win1 = 32 + lane < n_w ? stage_id(32 + lane) : -1;
+  int win0 = lane < n_w ? stage_id(lane, 0) : -1;
+  int win1 = 32 + lane < n_w ? stage_id(32 + lane, 0) : -1;
+  int win0b = kTwo && lane < n_w ? stage_id(lane, 1) : -1;
+  int win1b = kTwo && 32 + lane < n_w ? stage_id(32 + lane, 1) : -1;
 
   auto issue = [&](int k) {
     if (k - win_base >= 32) {
       win0 = win1;
       win_base += 32;
-      win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane) : -1;
+      win1 = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane, 0) : -1;
+      if constexpr (kTwo) {
+        win0b = win1b;
+        win1b = win_base + 32 + lane < n_w ? stage_id(win_base + 32 + lane, 1) : -1;
+      }
     }
     // After the rotation above, k - win_base < 32: read win0 only.  (Naming win1
     // here would make the shuffle wait for the window load just issued.)
     const int id = __shfl_sync(kFull, win0, k - win_base);
+    const int id_b = kTwo ? __shfl_sync(kFull, win0b, k - win_base) : 0;
+    // The L2 prefetch of stage k + kPrefetch (from the ring's second slot on; the
+    // prologue prefetches the first ones).  Its id is in window 1 only for the last
+    // stages before a rotation, long after that window was loaded.
+    int id_pf = -1;
+    if (kPrefetch > 0 && k >= C::kStages && k + kPrefetch < n_w) {
+      const int idx = k + kPrefetch - win_base;
+      id_pf = idx < 32 ? __shfl_sync(kFull, win0, idx) : __shfl_sync(kFull, win1, idx - 32);
+    }
     if (lane == 0) {
+      if (id_pf >= 0 && id_pf < p.num_blocks)  // a bad id is flagged at its load
+        C::prefetch_stage(&tmK, &tmV, kvh,
+                          id_pf * p.bs + (t_begin + (warp + kWarps * (k + kPrefetch)) * kStageTokens) % p.bs);
       const int s = k % C::kStages;
       const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
-      int row;
-      if (id < 0 || id >= p.num_blocks) {
-        flag_error(PKV_DEVERR_BLOCK_ID);
-        row = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
-      } else {
-        row = id * p.bs + t0 % p.bs;
-      }
+      const int oob = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
+      auto row_of = [&](int id_, int t) -> int {
+        if (id_ < 0 || id_ >= p.num_blocks) {
+          flag_error(PKV_DEVERR_BLOCK_ID);
+          return oob;
+        }
+        return id_ * p.bs + t % p.bs;
+      };
       mbar_arrive_expect_tx(&wbar[s], C::kStageBytes);
-      C::load_stage(ring + s * C::kStageBytes, &tmK, &tmV, &wbar[s], kvh, row, pol);
+      if constexpr (kTwo) {
+        // No tokens in the second half: a zero box, not a table read.
+        const int row1 = t0 + 8 < t_end ? row_of(id_b, t0 + 8) : oob;
+        C::load_stage_halves(ring + s * C::kStageBytes, &tmK, &tmV, &wbar[s], kvh,
+                             row_of(id, t0), row1, pol);
+      } else {
+        C::load_stage(ring + s * C::kStageBytes, &tmK, &tmV, &wbar[s], kvh, row_of(id, t0), pol);
+      }
     }
   };
 
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
   for (int k = 0; k < n_pro; ++k) issue(k);
+  if (kPrefetch > 0) {  // stages kStages .. kStages + kPrefetch - 1 (window 0)
+    static_assert(C::kStages + kPrefetch <= 32 || kPrefetch == 0, "prefetched stages lie in window 0");
+    const int k = C::kStages + lane;
+    const int id_pf = __shfl_sync(kFull, win0, k & 31);
+    if (lane < kPrefetch && k < n_w && id_pf >= 0 && id_pf < p.num_blocks)
+      C::prefetch_stage(&tmK, &tmV, kvh,
+                        id_pf * p.bs + (t_begin + (warp + kWarps * k) * kStageTokens) % p.bs);
+  }
 
   C c;
   c.init(p, b, kvh, lane);
@@ -755,9 +915,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
     const int n_valid = min(kStageTokens, t_end - t0);
-    c.consume(ring + s * C::kStageBytes, n_valid, lane);
-    __syncwarp();
-    if (k + C::kStages < n_w) issue(k + C::kStages);
+    c.consume(ring + s * C::kStageBytes, n_valid, lane, [&] {
+      if (k + C::kStages < n_w) issue(k + C::kStages);
+    });
   }
 
   // Merge the warps' states (each in its own, now idle, ring).

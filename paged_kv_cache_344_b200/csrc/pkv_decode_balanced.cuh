@@ -222,9 +222,10 @@ __global__ void __launch_bounds__(kWarps * 32)
           mbar_wait_bounded(&wbar[(kbase + j) % NS], ((kbase + j) / NS) & 1u);
         return;
       }
-      c.consume(ring + (kk % NS) * C::kStageBytes, min(kStageTokens, L - st * kStageTokens), lane);
-      __syncwarp();
-      if (k + NS < n) issue(k + NS);
+      c.consume(ring + (kk % NS) * C::kStageBytes, min(kStageTokens, L - st * kStageTokens), lane,
+                [&] {
+                  if (k + NS < n) issue(k + NS);
+                });
       ++st;
       ++pos;
       if (st < nst && pos < p_end) continue;

@@ -18,7 +18,7 @@
 // with a log-sum-exp rescale.  The result is the same softmax attention.
 //
 // Robustness: the prefix used for a group is shortened to one token less than
-// the shortest member and rounded down to 16 tokens; a prefix piece checks that
+// the shortest member and rounded down to whole blocks; a prefix piece checks that
 // every member's table entries for its blocks equal the first member's.  A
 // mismatch, or group offsets that do not cover the batch, flags
 // PKV_DEVERR_PREFIX (results are then unreliable; memory stays in bounds).
@@ -51,15 +51,17 @@ __device__ __forceinline__ int shared_len(const DecodeParams& d, int b) {
   return L < 0 ? 0 : (L > cap ? cap : L);
 }
 
-// Prefix actually shared by group g: short of every member's newest token (which
-// a fused step writes), whole stages.
+// Prefix actually shared by group g: short of every member's newest token, and
+// whole blocks (block_size is a multiple of the 16-token stage).  So no block of
+// the prefix is the one that receives a member's new token, which a fused step
+// rewrites (copy-on-write copy and the new row) while prefix pieces read.
 __device__ __forceinline__ int group_prefix(const SharedParams& s, int g, int lo, int hi) {
   int plen = s.prefix_lens[g];
   int minL = 0x7fffffff;
   for (int b = lo; b < hi; ++b) minL = min(minL, shared_len(s.d, b) - 1);
   if (hi <= lo) minL = 0;
   plen = max(0, min(plen, minL));
-  return plen & ~(kStageTokens - 1);
+  return plen / s.d.bs * s.d.bs;
 }
 
 // Group offset g clamped into [0, B]: offsets are caller data, and no value of
@@ -250,9 +252,9 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
       break;
     }
     const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
-    c.consume(ring + st * C::kStageBytes, min(kStageTokens, t_end - t0), lane);
-    __syncwarp();
-    if (k + C::kStages < n_w) issue(k + C::kStages);
+    c.consume(ring + st * C::kStageBytes, min(kStageTokens, t_end - t0), lane, [&] {
+      if (k + C::kStages < n_w) issue(k + C::kStages);
+    });
   }
 
   // Merge the warps; each row n = member * G + head goes to its sequence.
@@ -372,10 +374,49 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     if (threadIdx.x == 0) flag_error(PKV_DEVERR_PREFIX);
     members = mc;
   }
-  const int plen = group_prefix(s, g, lo, hi);  // whole stages
+  const int plen = group_prefix(s, g, lo, hi);  // whole blocks
+  uint8_t* ring = smem + warp * kRing;
+  uint64_t* wbar = bars + warp * C::kStages;
+  if (lane == 0) {
+    prefetch_tensormap(&tmK);
+    prefetch_tensormap(&tmV);
+#pragma unroll
+    for (int st = 0; st < C::kStages; ++st) mbar_init(&wbar[st], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t pol = l2_policy_evict_first();
+  // Stage meta words (valid tokens | member << 5 | every-row flag << 10), filed by
+  // lane 0 beside the stage's slot when it loads the stage.
+  __shared__ int s_meta[W][C::kStages];
+  // This warp's first stages (warp, warp + W, ...) that lie in the shared prefix
+  // need nothing but the first member's table row: their loads start before the
+  // fused step's writes and the set-up below (those writes never touch a prefix
+  // block, which ends before every member's newest token and on a block boundary).
+  int n_early = 0;
+  {
+    const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
+    const int n_pre0 = plen / kStageTokens;
+#pragma unroll
+    for (int kk = 0; kk < C::kStages; ++kk) {
+      const int k = warp + W * kk;
+      if (k >= n_pre0) break;
+      if (lane == 0) {
+        const int t0 = k * kStageTokens;
+        const int id = r0[t0 / p.bs];
+        int row = p.num_blocks * p.bs;  // past the pool: TMA fills zeros
+        if (id < 0 || id >= p.num_blocks) flag_error(PKV_DEVERR_BLOCK_ID);
+        else row = id * p.bs + t0 % p.bs;
+        s_meta[warp][kk] = kStageTokens | (1 << 10);
+        mbar_arrive_expect_tx(&wbar[kk], C::kStageBytes);
+        C::load_stage(ring + kk * C::kStageBytes, &tmK, &tmV, &wbar[kk], kvh, row, pol);
+      }
+      ++n_early;
+    }
+  }
   if (p.k_new != nullptr) {
     // Fused step: every member's new token (after any copy-on-write of its block)
-    // before anything is read.
+    // before anything else is read.
     for (int i = 0; i < members; ++i) {
       const int L = shared_len(p, lo + i);
       if (L > 0) fused_append<T, D>(p, lo + i, kvh, L);
@@ -420,23 +461,9 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   // This warp takes the CTA's stages warp, warp + W, ...
   const int first = warp, stride = W;
   const int n_w = n_all > first ? (n_all - first + stride - 1) / stride : 0;
-  uint8_t* ring = smem + warp * kRing;
-  uint64_t* wbar = bars + warp * C::kStages;
-  if (lane == 0) {
-    prefetch_tensormap(&tmK);
-    prefetch_tensormap(&tmV);
-#pragma unroll
-    for (int st = 0; st < C::kStages; ++st) mbar_init(&wbar[st], 1);
-    fence_mbar_init();
-  }
-  __syncwarp();
-  const uint64_t pol = l2_policy_evict_first();
   // The warp's stages win_base .. win_base + 63 are resolved ahead, one per lane
   // of two windows: the TMA row of the stage's 16 tokens (past the pool, so
-  // that TMA fills zeros, for a block id out of range) and its meta word (valid
-  // tokens | member << 5 | every-row flag << 10).  Lane 0 files the meta word of
-  // each stage it loads in s_meta beside the stage's slot.
-  __shared__ int s_meta[W][C::kStages];
+  // that TMA fills zeros, for a block id out of range) and its meta word.
   auto stage_info = [&](int kk, int& meta) -> int {
     int i, t0, nv;
     const bool all_rows = stage_of(first + stride * kk, i, t0, nv);
@@ -460,16 +487,33 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     }
     const int row = __shfl_sync(kFull, win0, kk - win_base);  // kk - win_base < 32 here
     const int meta = __shfl_sync(kFull, wm0, kk - win_base);
+    // The L2 prefetch of stage kk + kPrefetchStages (from the ring's second slot on;
+    // the prologue prefetches the first ones).  Its row is in window 1 only for the
+    // last stages before a rotation, long after that window was loaded.
+    int pf_row = -1;
+    if (kPrefetchStages > 0 && kk >= C::kStages && kk + kPrefetchStages < n_w) {
+      const int idx = kk + kPrefetchStages - win_base;
+      pf_row = idx < 32 ? __shfl_sync(kFull, win0, idx) : __shfl_sync(kFull, win1, idx - 32);
+    }
     if (lane == 0) {
       const int st = kk % C::kStages;
       s_meta[warp][st] = meta;
       mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
       C::load_stage(ring + st * C::kStageBytes, &tmK, &tmV, &wbar[st], kvh, row, pol);
+      // (a row past the pool stands for a bad block id: nothing to prefetch)
+      if (pf_row >= 0 && pf_row < p.num_blocks * p.bs) C::prefetch_stage(&tmK, &tmV, kvh, pf_row);
     }
     __syncwarp();  // the meta word is seen by every lane before the stage is consumed
   };
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
-  for (int kk = 0; kk < n_pro; ++kk) issue(kk);
+  for (int kk = n_early; kk < n_pro; ++kk) issue(kk);  // the early ones are in flight
+  if (kPrefetchStages > 0) {  // stages kStages .. kStages + kPrefetchStages - 1 (window 0)
+    static_assert(C::kStages + kPrefetchStages <= 32, "prefetched stages lie in window 0");
+    const int kk = C::kStages + lane;
+    const int r = __shfl_sync(kFull, win0, kk & 31);
+    if (lane < kPrefetchStages && kk < n_w && r < p.num_blocks * p.bs)
+      C::prefetch_stage(&tmK, &tmV, kvh, r);
+  }
 
   C c;
   c.init_gather(p, lo, members, kvh, lane);
@@ -484,12 +528,13 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     }
     const int meta = s_meta[warp][st];
     const int nv = meta & 31, r0 = ((meta >> 5) & 31) * G;
+    auto refill = [&] {
+      if (kk + C::kStages < n_w) issue(kk + C::kStages);
+    };
     if (meta >> 10)  // every member's rows score it
-      c.consume(ring + st * C::kStageBytes, nv, lane);
+      c.consume(ring + st * C::kStageBytes, nv, lane, refill);
     else
-      c.consume_rows(ring + st * C::kStageBytes, nv, lane, r0, r0 + G);
-    __syncwarp();
-    if (kk + C::kStages < n_w) issue(kk + C::kStages);
+      c.consume_rows(ring + st * C::kStageBytes, nv, lane, r0, r0 + G, refill);
   }
 
   // Merge the warps; each row n = member * G + head goes to its sequence.  The
@@ -548,7 +593,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
 
 // One CTA of W warps per (group, KV head): group_piece with consumer C (16 rows).
 template <class C, int D, int W>
-__global__ void __launch_bounds__(W * 32)
+__global__ void __launch_bounds__(W * 32, D <= 128 ? 2 : 1)
     paged_decode_group_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
                               const __grid_constant__ CUtensorMap tmV) {
   extern __shared__ uint8_t smem_raw[];

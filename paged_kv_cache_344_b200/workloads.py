@@ -249,8 +249,8 @@ def make(name: str, seed: int | None = None, scale_down: int = 1, block_size: in
         else:
             shared = np.full(n_groups, prefix)
             L = prefix + rng.integers(0, 256 // s + 1, size=B)
-        return _build(name, "bf16", B, 32, 8, 128, 16, L, seed, rng, groups=groups,
-                      shared_tokens=shared)
+        return _build(name, "bf16", B, 32, 8, 128, block_size or 16, L, seed, rng,
+                      groups=groups, shared_tokens=shared)
     raise KeyError(name)
 
 
@@ -347,6 +347,61 @@ def device_tensors(wl: Workload, device, seed_offset: int = 0) -> dict:
             c[i:j] = randn((j - i, bs, Hkv, D))
         c[invalid] = float("nan")
         out[key] = c
+    return out
+
+
+def valid_post(wl: Workload) -> np.ndarray:
+    """bool [NB, bs]: the slots that hold a token after the step (the pre-step tokens and
+    every sequence's new token)."""
+    v = wl.valid_pre.copy()
+    for s_ in wl.slot_mapping:
+        if s_ >= 0:
+            v[int(s_) // wl.bs, int(s_) % wl.bs] = True
+    return v
+
+
+def compact_sample(wl: Workload, n_seq: int, k_cache=None, v_cache=None, seed_offset: int = 0):
+    """The post-step decode inputs of sequences 0..n_seq-1 over a compact pool holding only
+    the blocks they use (a shared block once), with their block tables renumbered.
+
+    With ``k_cache``/``v_cache`` (torch tensors of the full pool, e.g. on the device after
+    the step), the blocks are gathered from them; otherwise they are drawn here (seeded
+    N(0,1), NaN in slots that hold no token).  Returns NumPy arrays (uint16 bf16 bits or
+    float32): q (drawn here unless the caller overrides it), k_cache, v_cache,
+    block_tables, seq_lens."""
+    n_seq = max(1, min(int(n_seq), wl.B))
+    lens = wl.seq_lens_post[:n_seq]
+    ids, remap = [], {}
+    tables = np.full((n_seq, max(1, max(_ceil_div(int(L), wl.bs) for L in lens))), -1, np.int32)
+    for b in range(n_seq):
+        for j in range(_ceil_div(int(lens[b]), wl.bs)):
+            pid = int(wl.block_tables[b, j])
+            if pid not in remap:
+                remap[pid] = len(ids)
+                ids.append(pid)
+            tables[b, j] = remap[pid]
+    ids = np.asarray(ids, dtype=np.int64)
+    rng = np.random.default_rng(wl.seed * 7919 + 29 + seed_offset)
+    shape = (len(ids), wl.bs, wl.Hkv, wl.D)
+    if k_cache is not None:
+        import torch
+        sel = torch.from_numpy(ids).to(k_cache.device)
+        out = {}
+        for key, c in (("k_cache", k_cache), ("v_cache", v_cache)):
+            t = c.index_select(0, sel).cpu().contiguous()
+            out[key] = t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 \
+                else t.numpy()
+    else:
+        invalid = ~valid_post(wl)[ids]
+        out = {}
+        for key in ("k_cache", "v_cache"):
+            x = rng.standard_normal(shape, dtype=np.float32)
+            x[invalid] = np.nan
+            out[key] = _to_bf16_bits(x) if wl.dtype == "bf16" else x
+    q = rng.standard_normal((n_seq, wl.Hq, wl.D), dtype=np.float32)
+    out["q"] = _to_bf16_bits(q) if wl.dtype == "bf16" else q
+    out["block_tables"] = tables
+    out["seq_lens"] = np.ascontiguousarray(lens, dtype=np.int32)
     return out
 
 

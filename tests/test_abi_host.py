@@ -93,7 +93,8 @@ def test_decode_rejects_bad_arguments(lib):
     assert _decode(lib, part=24) == ERR_ARG
     assert _decode(lib, D=96) == ERR_UNSUP
     assert _decode(lib, D=256, dt=1) == ERR_UNSUP
-    assert _decode(lib, bs=8) == ERR_UNSUP
+    assert _decode(lib, bs=24) == ERR_UNSUP  # 8, or a multiple of 16
+    assert _decode(lib, bs=4) == ERR_UNSUP
     assert _decode(lib, Hq=64, Hkv=2) == ERR_UNSUP  # G = 32
     assert _decode(lib, msl=8 * 16 + 1) == ERR_RANGE
     assert _decode(lib, nb=(1 << 31) // 16) == ERR_RANGE
@@ -103,6 +104,24 @@ def test_decode_rejects_bad_arguments(lib):
     assert _decode(lib, msl=128, part=16, ws=FAKE + 16, wsb=1 << 20) == ERR_WS  # misaligned
     # an empty batch is a no-op that succeeds without touching the device
     assert _decode(lib, B=0) == 0
+
+
+@host_only
+def test_contiguous_control_rejects_bad_arguments(lib):
+    def c(**kw):
+        a = dict(out=FAKE, k=FAKE, msl=100, stride=128, B=2, Hq=8, Hkv=2, D=128, dt=0, part=0)
+        a.update(kw)
+        return lib.paged_attention_decode_contiguous(
+            a["out"], FAKE, a["k"], FAKE, FAKE, a["msl"], a["stride"], a["B"], a["Hq"], a["Hkv"],
+            a["D"], 0.1, a["dt"], a["part"], None, 0, None)
+    assert c(stride=99) == ERR_ARG  # a row stride shorter than the longest sequence
+    assert c(stride=0) == ERR_ARG
+    assert c(out=None) == ERR_ARG
+    assert c(k=FAKE + 8) == ERR_ARG
+    assert c(dt=1) == ERR_UNSUP  # the control runs the bf16 tensor-core kernel only
+    assert c(D=96) == ERR_UNSUP
+    assert c(msl=128, part=16) == ERR_WS  # split into partitions without a workspace
+    assert c(B=0) == 0
 
 
 @host_only

@@ -120,3 +120,25 @@ def test_stalled_wait_gives_up_and_attention_stands_down():
     _, _, ref = oracle_step(wl, host)
     assert_attention_close(widen(out), ref, wl.dtype, "fused step after clearing")
     assert pkv.device_errors() == 0
+
+
+def test_workspace_zero_fill_restores_it_after_a_timeout():
+    """A launch stopped by a timeout can leave partition tickets non-zero in its workspace
+    (its CTAs that stopped early took none).  The documented remedy is to zero-fill the
+    workspace before its next use; this plants such leftover tickets, applies the remedy
+    and checks that the decode is exact again."""
+    pkv.device_errors(clear=True)
+    wl = workloads.make("long", scale_down=16)
+    host = workloads.host_tensors(wl)
+    dev = device_inputs(wl, host)
+    P = 64
+    ws = workspace_for(wl, P)
+    units = wl.B * wl.Hkv
+    ws[:4 * units].view(torch.int32).fill_(3)  # what a stopped launch may leave behind
+    ws.zero_()  # the remedy: zero-fill before the next use
+    out = gpu_step(wl, dev, partition_size=P, workspace=ws, fused=True)
+    torch.cuda.synchronize()
+    _, _, ref = oracle_step(wl, host)
+    assert_attention_close(widen(out), ref, wl.dtype, "after zero-filling the workspace")
+    assert int(ws[:4 * units].view(torch.int32).abs().sum()) == 0  # tickets back at zero
+    assert pkv.device_errors() == 0

@@ -107,3 +107,21 @@ def test_fused_shared_prefix_random_groups():
     assert to_host_bits(dev["k_cache"]).tobytes() == kc.tobytes()
     assert_attention_close(widen(out), ref, wl.dtype, "random groups")
     assert pkv.device_errors() == 0
+
+
+@pytest.mark.parametrize("shared", [False, True])
+@pytest.mark.parametrize("P", [16, 48])
+def test_fused_step_partition_shorter_than_block(P, shared):
+    """Blocks of 32 tokens with partitions of 16 or 48: the step copies (copy-on-write) and
+    rewrites the block of each new token, so the library rounds the partition up to whole
+    blocks and no other partition reads that block while it is rewritten."""
+    wl = workloads.make("share_fork", scale_down=4, block_size=32)
+    assert len(wl.cow_pairs) > 0 and wl.bs == 32
+    host = workloads.host_tensors(wl)
+    dev = device_inputs(wl, host)
+    out = gpu_step(wl, dev, partition_size=P, fused=True, shared=shared)
+    kc, vc, ref = oracle_step(wl, host)
+    assert to_host_bits(dev["k_cache"]).tobytes() == kc.tobytes()
+    assert to_host_bits(dev["v_cache"]).tobytes() == vc.tobytes()
+    assert_attention_close(widen(out), ref, wl.dtype, f"bs=32 P={P} shared={shared}")
+    assert pkv.device_errors() == 0

@@ -5,8 +5,8 @@ example a host whose device memory is entirely owned by its own pool, or a servi
 that must not call cudaMalloc mid-step because the call may synchronise the device).  It
 keeps its split-partition scratch in a fixed array inside the library.  These tests call
 it through the C ABI and check that two calls in a row give what the regular entry point
-gives, within the parity tolerance, and that sizes needing more scratch than the array
-holds are rejected.  They set up everything they use, so they pass alone in a fresh
+gives, and what the fp64 oracle gives (with either work split), within the parity
+tolerance, and that sizes needing more scratch than the array holds are rejected.  They set up everything they use, so they pass alone in a fresh
 process as well as after the rest of the suite.
 """
 import ctypes
@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_344_b200 as pkv
 from paged_kv_cache_344_b200 import workloads
 from gpu_util import assert_attention_close, device_inputs, widen, workspace_for
@@ -56,6 +57,31 @@ def test_noalloc_matches_regular_entry_point(name, sd, P):
         assert _noalloc_raw(out, d, wl, wl.max_seq_len, P) == pkv.PKV_OK
         torch.cuda.synchronize()
         assert_attention_close(widen(out), expect, wl.dtype, f"{name} P={P} call {call}")
+    assert pkv.device_errors() == 0
+
+
+@pytest.mark.parametrize("split", ["fixed", "balanced"])
+def test_noalloc_matches_oracle(split):
+    """The allocation-free decode against the fp64 oracle directly, with the library's
+    default split and with the work-balanced split (whose scratch layout differs)."""
+    pkv.device_errors(clear=True)
+    wl = workloads.make("long", scale_down=16)
+    host = workloads.host_tensors(wl)
+    d = device_inputs(wl, host)
+    pkv.paged_kv_write(d["k_new"], d["v_new"], d["k_cache"], d["v_cache"], d["slot_mapping"])
+    kc, vc = host["k_cache"].copy(), host["v_cache"].copy()
+    assert oracle.kv_write(host["k_new"], host["v_new"], kc, vc, wl.slot_mapping) == 0
+    ref = oracle.paged_decode(host["q"], kc, vc, wl.block_tables, wl.seq_lens_post, wl.scale)
+    old = pkv.set_decode_split(pkv.PKV_SPLIT_BALANCED if split == "balanced"
+                               else pkv.PKV_SPLIT_FIXED)
+    try:
+        for call in range(2):
+            out = torch.full_like(d["q"], float("nan"))
+            assert _noalloc_raw(out, d, wl, wl.max_seq_len, 0) == pkv.PKV_OK
+            torch.cuda.synchronize()
+            assert_attention_close(widen(out), ref, wl.dtype, f"{split} call {call}")
+    finally:
+        pkv.set_decode_split(old)
     assert pkv.device_errors() == 0
 
 
