@@ -333,7 +333,8 @@ struct SimtConsumer {
 #define PKV_MMA_STAGES_D128 2
 #endif
 
-template <int D, int NT, int STAGES = (D <= 64 ? 6 : (D <= 128 ? PKV_MMA_STAGES_D128 : 2))>
+template <int D, int NT, int STAGES = (D <= 64 ? 6 : (D <= 128 ? PKV_MMA_STAGES_D128 : 2)),
+          bool EARLY = (D <= 128 && NT == 1)>
 struct MmaConsumer {
   static constexpr int SUB = D / 64;
   static constexpr int kSubBytes = kStageTokens * 128;
@@ -346,8 +347,10 @@ struct MmaConsumer {
   static constexpr bool kSwizzle = true;
   static constexpr bool kCanPrefetch = true;
   // V fragments held in registers so that the stage is released before the
-  // softmax (D <= 128; at D = 256 they would not fit next to O).
-  static constexpr bool kEarly = D <= 128;
+  // softmax.  By default for one 8-row head tile up to D = 128: with two tiles (16
+  // query rows) or D = 256 the extra registers cost a resident CTA per SM (or
+  // spill), and measured on B200 the early release gains nothing there.
+  static constexpr bool kEarly = EARLY;
 
   uint32_t qf[NT][KS][2];
   float m[NT][2], l[NT][2];
