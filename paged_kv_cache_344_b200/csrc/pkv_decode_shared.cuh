@@ -334,6 +334,64 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
   }
 }
 
+// Fused step of a group CTA (one KV head): every member's copy-on-write copy and
+// new token row in one pass over all members.  Each element is written once: the
+// copy leaves out the row that the new token fills, so no thread waits for another,
+// and no member ever reads a row that another member is writing (in a fork the last
+// holder writes its token into the block the others copy from, at the row they
+// leave out).  The result equals copy_blocks then paged_kv_write.  Warp 0 resolves
+// each member's blocks first (s_dst < 0: nothing to write).
+template <typename T, int D>
+__device__ __forceinline__ void group_append(const DecodeParams& p, int lo, int members, int kvh,
+                                             int* s_dst, int* s_src, int* s_row) {
+  if (threadIdx.x < (unsigned)members) {  // members <= 16
+    const int b = lo + (int)threadIdx.x;
+    const int L = shared_len(p, b);
+    int dst = -1, src = -1, row = 0;
+    if (L > 0) {
+      const int t = L - 1;
+      const int id = p.block_tables[(size_t)b * p.max_blocks + t / p.bs];
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PKV_DEVERR_BLOCK_ID);
+      } else {
+        dst = id;
+        row = t % p.bs;
+        const int c = p.cow_src != nullptr ? p.cow_src[b] : -1;
+        if (c >= p.num_blocks) flag_error(PKV_DEVERR_COPY);
+        else if (c >= 0 && c != id) src = c;
+      }
+    }
+    s_dst[threadIdx.x] = dst;
+    s_src[threadIdx.x] = src;
+    s_row[threadIdx.x] = row;
+  }
+  __syncthreads();
+  constexpr int kVec = D * (int)sizeof(T) / 16;  // 16-byte vectors per head row
+  const size_t row_vec = (size_t)p.Hkv * kVec;    // per token row (all heads)
+  uint4* kc = reinterpret_cast<uint4*>(p.k_cache_w);
+  uint4* vc = reinterpret_cast<uint4*>(p.v_cache_w);
+  const uint4* kn = reinterpret_cast<const uint4*>(p.k_new);
+  const uint4* vn = reinterpret_cast<const uint4*>(p.v_new);
+  const int per = (p.bs + 1) * kVec;  // per member: the block's rows, then the new row
+  for (int x = threadIdx.x; x < members * per; x += blockDim.x) {
+    const int i = x / per, r = (x % per) / kVec, c = x % kVec;
+    const int dst = s_dst[i];
+    if (dst < 0) continue;
+    if (r == p.bs) {
+      const size_t d_o = ((size_t)dst * p.bs + s_row[i]) * row_vec + (size_t)kvh * kVec + c;
+      const size_t so = ((size_t)(lo + i) * p.Hkv + kvh) * kVec + c;
+      kc[d_o] = kn[so];
+      vc[d_o] = vn[so];
+    } else if (s_src[i] >= 0 && r != s_row[i]) {
+      const size_t so = ((size_t)s_src[i] * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
+      const size_t d_o = ((size_t)dst * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
+      kc[d_o] = kc[so];
+      vc[d_o] = vc[so];
+    }
+  }
+  fence_proxy_async_global();
+}
+
 // One CTA for a whole group and one KV head, when the group's members fit the
 // 16 query rows of one MMA (members <= 16 / G).  The CTA's stages are the
 // shared prefix's (scored for every member's rows) followed by each member's
@@ -417,10 +475,8 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   if (p.k_new != nullptr) {
     // Fused step: every member's new token (after any copy-on-write of its block)
     // before anything else is read.
-    for (int i = 0; i < members; ++i) {
-      const int L = shared_len(p, lo + i);
-      if (L > 0) fused_append<T, D>(p, lo + i, kvh, L);
-    }
+    __shared__ int s_adst[kMaxMembers], s_asrc[kMaxMembers], s_arow[kMaxMembers];
+    group_append<T, D>(p, lo, members, kvh, s_adst, s_asrc, s_arow);
     __syncthreads();
   }
   if (threadIdx.x == 0) {
