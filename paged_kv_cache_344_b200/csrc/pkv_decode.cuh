@@ -33,14 +33,6 @@ namespace pkv {
 
 constexpr int kStageTokens = 16;  // tokens per TMA box / pipeline stage
 
-// Stages a warp prefetches into L2 ahead of its ring (tensor-core consumers).  A
-// warp keeps only kStages stages in flight into shared memory; the L2 prefetches
-// of the next ones put more bytes in flight without holding shared memory, so the
-// ring's own loads hit L2.
-#ifndef PKV_PREFETCH_STAGES
-#define PKV_PREFETCH_STAGES 0
-#endif
-constexpr int kPrefetchStages = PKV_PREFETCH_STAGES;
 constexpr int kWarps = 4;         // consumer warps per CTA
 constexpr uint32_t kFull = 0xffffffffu;
 
@@ -157,9 +149,6 @@ struct SimtConsumer {
   static constexpr int kStages = ROWB <= 128 ? 6 : (ROWB <= 256 ? 3 : 2);
   static constexpr int GP = GMAX;
   static constexpr bool kSwizzle = false;
-  static constexpr bool kCanPrefetch = false;  // (3-D maps; no L2 prefetch path)
-  static __device__ __forceinline__ void prefetch_stage(const CUtensorMap*, const CUtensorMap*,
-                                                        int, int) {}
   static_assert(LPT >= 1 && LPT <= 32 && TPI * LPT == 32, "bad lane split");
 
   float qv[GMAX][2][EPC];
@@ -345,7 +334,6 @@ struct MmaConsumer {
   static constexpr int MT = D / 16;
   static constexpr int GP = 8 * NT;
   static constexpr bool kSwizzle = true;
-  static constexpr bool kCanPrefetch = true;
   // V fragments held in registers so that the stage is released before the
   // softmax.  By default for one 8-row head tile up to D = 128: with two tiles (16
   // query rows) or D = 256 the extra registers cost a resident CTA per SM (or
@@ -421,13 +409,6 @@ struct MmaConsumer {
                                                     int kvh, int row, uint64_t pol) {
     tma_load_4d(st, tk, bar, 0, row, 0, kvh, pol);
     tma_load_4d(st + kTileBytes, tv, bar, 0, row, 0, kvh, pol);
-  }
-
-  // An L2 prefetch of the stage's K and V boxes (a later load_stage finds them there).
-  static __device__ __forceinline__ void prefetch_stage(const CUtensorMap* tk,
-                                                        const CUtensorMap* tv, int kvh, int row) {
-    tma_prefetch_4d(tk, 0, row, 0, kvh);
-    tma_prefetch_4d(tv, 0, row, 0, kvh);
   }
 
   // Blocks of 8 tokens: the maps' box is {64, 8, 1, 1}, and each 64-dim sub-tile is
@@ -836,7 +817,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   // Physical ids of this warp's stages win_base .. win_base+63 (one per lane, two
   // windows; with 8-token blocks a second pair for the stages' second halves).
   constexpr bool kTwo = LAYOUT == kLayoutPaged8;
-  constexpr int kPrefetch = C::kCanPrefetch && !kTwo ? kPrefetchStages : 0;
   int win_base = 0;
   int win0 = lane < n_w ? stage_id(lane, 0) : -1;
   int win1 = 32 + lane < n_w ? stage_id(32 + lane, 0) : -1;
@@ -857,18 +837,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     // here would make the shuffle wait for the window load just issued.)
     const int id = __shfl_sync(kFull, win0, k - win_base);
     const int id_b = kTwo ? __shfl_sync(kFull, win0b, k - win_base) : 0;
-    // The L2 prefetch of stage k + kPrefetch (from the ring's second slot on; the
-    // prologue prefetches the first ones).  Its id is in window 1 only for the last
-    // stages before a rotation, long after that window was loaded.
-    int id_pf = -1;
-    if (kPrefetch > 0 && k >= C::kStages && k + kPrefetch < n_w) {
-      const int idx = k + kPrefetch - win_base;
-      id_pf = idx < 32 ? __shfl_sync(kFull, win0, idx) : __shfl_sync(kFull, win1, idx - 32);
-    }
     if (lane == 0) {
-      if (id_pf >= 0 && id_pf < p.num_blocks)  // a bad id is flagged at its load
-        C::prefetch_stage(&tmK, &tmV, kvh,
-                          id_pf * p.bs + (t_begin + (warp + kWarps * (k + kPrefetch)) * kStageTokens) % p.bs);
       const int s = k % C::kStages;
       const int t0 = t_begin + (warp + kWarps * k) * kStageTokens;
       const int oob = p.num_blocks * p.bs;  // entirely out of bounds: TMA fills zeros
@@ -893,14 +862,6 @@ __global__ void __launch_bounds__(kWarps * 32)
 
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
   for (int k = 0; k < n_pro; ++k) issue(k);
-  if (kPrefetch > 0) {  // stages kStages .. kStages + kPrefetch - 1 (window 0)
-    static_assert(C::kStages + kPrefetch <= 32 || kPrefetch == 0, "prefetched stages lie in window 0");
-    const int k = C::kStages + lane;
-    const int id_pf = __shfl_sync(kFull, win0, k & 31);
-    if (lane < kPrefetch && k < n_w && id_pf >= 0 && id_pf < p.num_blocks)
-      C::prefetch_stage(&tmK, &tmV, kvh,
-                        id_pf * p.bs + (t_begin + (warp + kWarps * k) * kStageTokens) % p.bs);
-  }
 
   C c;
   c.init(p, b, kvh, lane);

@@ -339,11 +339,11 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
 // copy leaves out the row that the new token fills, so no thread waits for another,
 // and no member ever reads a row that another member is writing (in a fork the last
 // holder writes its token into the block the others copy from, at the row they
-// leave out).  The result equals copy_blocks then paged_kv_write.  Warp 0 resolves
-// each member's blocks first (s_dst < 0: nothing to write).
-template <typename T, int D>
-__device__ __forceinline__ void group_append(const DecodeParams& p, int lo, int members, int kvh,
-                                             int* s_dst, int* s_src, int* s_row) {
+// leave out).  The result equals copy_blocks then paged_kv_write.  Each member's
+// blocks are resolved first (s_dst < 0: nothing to write).
+// Phase 1 (threads < members, before a CTA barrier): each member's blocks.
+__device__ __forceinline__ void group_append_resolve(const DecodeParams& p, int lo, int members,
+                                                     int* s_dst, int* s_src, int* s_row) {
   if (threadIdx.x < (unsigned)members) {  // members <= 16
     const int b = lo + (int)threadIdx.x;
     const int L = shared_len(p, b);
@@ -365,7 +365,13 @@ __device__ __forceinline__ void group_append(const DecodeParams& p, int lo, int 
     s_src[threadIdx.x] = src;
     s_row[threadIdx.x] = row;
   }
-  __syncthreads();
+}
+
+// Phase 2 (every thread, after that barrier): the copies and the new rows.
+template <typename T, int D>
+__device__ __forceinline__ void group_append_write(const DecodeParams& p, int lo, int members,
+                                                   int kvh, const int* s_dst, const int* s_src,
+                                                   const int* s_row) {
   constexpr int kVec = D * (int)sizeof(T) / 16;  // 16-byte vectors per head row
   const size_t row_vec = (size_t)p.Hkv * kVec;    // per token row (all heads)
   uint4* kc = reinterpret_cast<uint4*>(p.k_cache_w);
@@ -472,14 +478,13 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
       ++n_early;
     }
   }
-  if (p.k_new != nullptr) {
-    // Fused step: every member's new token (after any copy-on-write of its block)
-    // before anything else is read.
-    __shared__ int s_adst[kMaxMembers], s_asrc[kMaxMembers], s_arow[kMaxMembers];
-    group_append<T, D>(p, lo, members, kvh, s_adst, s_asrc, s_arow);
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) {
+  // Set-up: each member's stage count (s_cum) and, for a fused step, the blocks its
+  // new token goes to; then the fused step's writes (every member's new token after
+  // any copy-on-write of its block) land before any stage of own tokens is loaded.
+  const bool fused = p.k_new != nullptr;
+  __shared__ int s_adst[kMaxMembers], s_asrc[kMaxMembers], s_arow[kMaxMembers];
+  if (fused) group_append_resolve(p, lo, members, s_adst, s_asrc, s_arow);
+  if (threadIdx.x == blockDim.x - 1) {
     int cum = plen / kStageTokens;
     s_cum[0] = cum;
     for (int i = 0; i < members; ++i) {
@@ -490,6 +495,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     }
   }
   __syncthreads();
+  if (fused) group_append_write<T, D>(p, lo, members, kvh, s_adst, s_asrc, s_arow);
   {  // every member must hold the same physical blocks for the prefix
     const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
     const int nj = plen > 0 ? (plen - 1) / p.bs + 1 : 0;
@@ -498,6 +504,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
       if (p.block_tables[(size_t)b * p.max_blocks + j] != r0[j]) flag_error(PKV_DEVERR_PREFIX);
     }
   }
+  if (fused) __syncthreads();
   const int n_pre = s_cum[0], n_all = s_cum[members];
   // Stage k of the CTA: the member i whose table row it reads, its first token
   // and its valid tokens; true when every member's rows score it (a prefix stage,
@@ -543,33 +550,16 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     }
     const int row = __shfl_sync(kFull, win0, kk - win_base);  // kk - win_base < 32 here
     const int meta = __shfl_sync(kFull, wm0, kk - win_base);
-    // The L2 prefetch of stage kk + kPrefetchStages (from the ring's second slot on;
-    // the prologue prefetches the first ones).  Its row is in window 1 only for the
-    // last stages before a rotation, long after that window was loaded.
-    int pf_row = -1;
-    if (kPrefetchStages > 0 && kk >= C::kStages && kk + kPrefetchStages < n_w) {
-      const int idx = kk + kPrefetchStages - win_base;
-      pf_row = idx < 32 ? __shfl_sync(kFull, win0, idx) : __shfl_sync(kFull, win1, idx - 32);
-    }
     if (lane == 0) {
       const int st = kk % C::kStages;
       s_meta[warp][st] = meta;
       mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
       C::load_stage(ring + st * C::kStageBytes, &tmK, &tmV, &wbar[st], kvh, row, pol);
-      // (a row past the pool stands for a bad block id: nothing to prefetch)
-      if (pf_row >= 0 && pf_row < p.num_blocks * p.bs) C::prefetch_stage(&tmK, &tmV, kvh, pf_row);
     }
     __syncwarp();  // the meta word is seen by every lane before the stage is consumed
   };
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
   for (int kk = n_early; kk < n_pro; ++kk) issue(kk);  // the early ones are in flight
-  if (kPrefetchStages > 0) {  // stages kStages .. kStages + kPrefetchStages - 1 (window 0)
-    static_assert(C::kStages + kPrefetchStages <= 32, "prefetched stages lie in window 0");
-    const int kk = C::kStages + lane;
-    const int r = __shfl_sync(kFull, win0, kk & 31);
-    if (lane < kPrefetchStages && kk < n_w && r < p.num_blocks * p.bs)
-      C::prefetch_stage(&tmK, &tmV, kvh, r);
-  }
 
   C c;
   c.init_gather(p, lo, members, kvh, lane);

@@ -150,17 +150,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// Prefetch of one 4-D box into L2 (no shared memory, no barrier): a later TMA
-// load of the same box then finds it in L2.  No cluster multicast.
-__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2,
-                                                int c3) {
-  asm volatile(
-      "cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
 // L2 policy for data read exactly once (the K/V stream).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
