@@ -110,11 +110,13 @@ def test_fused_shared_prefix_random_groups():
 
 
 @pytest.mark.parametrize("shared", [False, True])
-@pytest.mark.parametrize("P", [16, 48])
+@pytest.mark.parametrize("P", [0, 16, 48])
 def test_fused_step_partition_shorter_than_block(P, shared):
     """Blocks of 32 tokens with partitions of 16 or 48: the step copies (copy-on-write) and
     rewrites the block of each new token, so the library rounds the partition up to whole
-    blocks and no other partition reads that block while it is rewritten."""
+    blocks and no other partition reads that block while it is rewritten.  P = 0 with the
+    shared-prefix step runs the one-CTA-per-group kernel, whose writes leave out the row
+    each new token fills when they copy a block."""
     wl = workloads.make("share_fork", scale_down=4, block_size=32)
     assert len(wl.cow_pairs) > 0 and wl.bs == 32
     host = workloads.host_tensors(wl)
