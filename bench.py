@@ -273,7 +273,8 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
     import paged_kv_cache_344_b200 as pkv
 
     dev_name = f"cuda:{local_rank}"
-    wl = workloads.make(name, block_size=args.block_size or None, contiguous=args.contiguous)
+    wl = workloads.make(name, block_size=args.block_size or None, contiguous=args.contiguous,
+                        dtype=args.dtype or None)
     dev = workloads.device_tensors(wl, dev_name, seed_offset=rank)
     meta = {
         "block_tables": torch.from_numpy(wl.block_tables).to(dev_name),
@@ -818,7 +819,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     wl = workloads.make(args.config, block_size=args.block_size or None,
-                        contiguous=args.contiguous)
+                        contiguous=args.contiguous, dtype=args.dtype or None)
     n_seq = oracle_sample_size(wl, args.cpu_budget_rows // max(args.steps, 1))
     sample = workloads.compact_sample(wl, n_seq)
     nw = max(1, n_seq // 8)  # warm-up: the first sequences of the same sample
@@ -883,6 +884,9 @@ def main():
                          "workloads, the plain decode otherwise)")
     ap.add_argument("--block-size", type=int, default=0,
                     help="override the workload's block size (block-size sweep)")
+    ap.add_argument("--dtype", choices=["", "bf16", "f32"], default="",
+                    help="element type override for the mha/gqa/long workloads (f32 runs the "
+                         "CUDA-core consumer)")
     ap.add_argument("--contiguous", action="store_true",
                     help="lay each sequence's blocks out consecutively (contiguous-cache control)")
     ap.add_argument("--step", choices=["separate", "fused"], default="fused",

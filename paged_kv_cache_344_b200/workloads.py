@@ -202,7 +202,7 @@ CONFIG_INDEX = {"tiny": 0, "tiny_post": 0, "mha": 1, "gqa16": 2, "gqa32": 2, "lo
 
 
 def make(name: str, seed: int | None = None, scale_down: int = 1, block_size: int | None = None,
-         contiguous: bool = False) -> Workload:
+         contiguous: bool = False, dtype: str | None = None) -> Workload:
     """Build a named workload.
 
     Full-size names: ``tiny`` (lengths are pre-step), ``tiny_post`` (lengths include the
@@ -210,7 +210,8 @@ def make(name: str, seed: int | None = None, scale_down: int = 1, block_size: in
     ``scale_down > 1`` divides the batch and the lengths for fast parity tests while keeping
     the head shapes, block size and length distribution.  ``block_size`` overrides the
     workload's block size; ``contiguous`` lays every sequence's blocks out consecutively
-    (a contiguous-cache control for the cost of the scattered placement).
+    (a contiguous-cache control for the cost of the scattered placement); ``dtype`` ("bf16"
+    or "f32") overrides the element type of the bf16 workloads.
     """
     kw = {"contiguous": contiguous}
     if seed is None:
@@ -225,18 +226,18 @@ def make(name: str, seed: int | None = None, scale_down: int = 1, block_size: in
     if name == "mha":
         B = max(64 // s, 2)
         L = rng.integers(128 // s, 2048 // s + 1, size=B)
-        return _build(name, "bf16", B, 40, 40, 128, block_size or 16, L, seed, rng, **kw)
+        return _build(name, dtype or "bf16", B, 40, 40, 128, block_size or 16, L, seed, rng, **kw)
     if name in ("gqa16", "gqa32"):
         bs = block_size or (16 if name == "gqa16" else 32)
         B = max(256 // s, 2)
         z = rng.standard_normal(B)
         L = np.clip(np.round(np.exp(math.log(1024) + 0.8 * z)), 16, 4096).astype(np.int64) // s
         L = np.maximum(L, 1)
-        return _build(name, "bf16", B, 32, 8, 128, bs, L, seed, rng, **kw)
+        return _build(name, dtype or "bf16", B, 32, 8, 128, bs, L, seed, rng, **kw)
     if name == "long":
         B = max(8 // s, 1)
         L = rng.integers(32768 // s, 131072 // s + 1, size=B)
-        return _build(name, "bf16", B, 64, 8, 128, block_size or 16, L, seed, rng, **kw)
+        return _build(name, dtype or "bf16", B, 64, 8, 128, block_size or 16, L, seed, rng, **kw)
     if name in ("share_fork", "share_tails"):
         n_groups, branches = max(32 // s, 1), 4
         B = n_groups * branches
