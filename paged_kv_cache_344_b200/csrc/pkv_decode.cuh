@@ -10,11 +10,15 @@
 // How (B200 design):
 //  * one CTA per (kvh, partition, b); the G query heads of a KV head share
 //    every K/V byte read, so the cache is read once per (b, kvh);
-//  * K/V arrive by TMA: a 3-D tensor map over [num_blocks*bs][Hkv][D] fetches
-//    one 16-token slab of one KV head per box; each consumer warp owns a ring
-//    of stages and refills it itself, so no CTA-wide barrier sits in the loop;
+//  * K/V arrive by TMA, one 16-token slab of one KV head per box (a 4-D map
+//    with the 128-byte swizzle for the tensor-core consumer, a 3-D map for the
+//    CUDA-core one; with 8-token blocks a stage is two 8-token boxes from two
+//    blocks); each consumer warp owns a ring of stages and refills it itself,
+//    so no CTA-wide barrier sits in the loop;
 //  * the block-table walk (the "pointer chase") is taken off the critical path:
-//    each warp keeps the physical ids of its next 32..64 stages in registers;
+//    each warp keeps the physical ids of its next 32..64 stages in registers.
+//    The unpaged control (kLayoutContig) reads [B][stride][Hkv][D] with no
+//    table at all, to measure what the walk costs;
 //  * online softmax in fp32 (running max and sum, exp2 with the scale folded
 //    into log2 units), per warp; warps and then partitions are merged with a
 //    log-sum-exp rescale;
@@ -32,7 +36,6 @@
 namespace pkv {
 
 constexpr int kStageTokens = 16;  // tokens per TMA box / pipeline stage
-
 constexpr int kWarps = 4;         // consumer warps per CTA
 constexpr uint32_t kFull = 0xffffffffu;
 
@@ -436,9 +439,9 @@ struct MmaConsumer {
   }
 
   // Consumes one stage; `release()` (warp-collective) is called as soon as the
-  // stage's shared memory has been read (K by the score MMAs, V into registers),
-  // so that the warp can refill the slot while it still computes the softmax and
-  // the P V product.
+  // stage's shared memory has been read: with kEarly after the score MMAs and the
+  // V fragments' loads into registers, so that the warp refills the slot while it
+  // still computes the softmax and the P V product; otherwise after the P V product.
   template <class Release>
   __device__ __forceinline__ void consume(uint8_t* st, int n_valid, int lane, Release&& release) {
     consume_impl<false>(st, n_valid, lane, 0, GP, release);
@@ -488,10 +491,9 @@ struct MmaConsumer {
 
     // V^T fragments (A operand of O^T += V^T P): lane (g, t) = (lane / 4, lane % 4)
     // holds dims (g, g + 8) of each 16-dim tile for tokens (2t, 2t + 1) in
-    // va[mt][0..1] and (2t + 8, 2t + 9) in va[mt][2..3].  Up to D = 128 they are
-    // read into registers here and the slot is released at once; at D = 256 the
-    // registers do not suffice, V is read during the P V product and the slot is
-    // released after it.
+    // va[mt][0..1] and (2t + 8, 2t + 9) in va[mt][2..3].  With kEarly all of them
+    // are read into registers here and the slot is released at once; otherwise
+    // each is read during the P V product and the slot is released after it.
     uint32_t va[kEarly ? MT : 1][4];
     auto load_v = [&](int mt, uint32_t (&a)[4]) {
       const int t = (mi >> 1) * 8 + rr;
