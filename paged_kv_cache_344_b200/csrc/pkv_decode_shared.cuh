@@ -339,62 +339,69 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
 // copy leaves out the row that the new token fills, so no thread waits for another,
 // and no member ever reads a row that another member is writing (in a fork the last
 // holder writes its token into the block the others copy from, at the row they
-// leave out).  The result equals copy_blocks then paged_kv_write.  Each member's
-// blocks are resolved first (s_dst < 0: nothing to write).
-// Phase 1 (threads < members, before a CTA barrier): each member's blocks.
-__device__ __forceinline__ void group_append_resolve(const DecodeParams& p, int lo, int members,
-                                                     int* s_dst, int* s_src, int* s_row) {
-  if (threadIdx.x < (unsigned)members) {  // members <= 16
-    const int b = lo + (int)threadIdx.x;
-    const int L = shared_len(p, b);
-    int dst = -1, src = -1, row = 0;
-    if (L > 0) {
-      const int t = L - 1;
-      const int id = p.block_tables[(size_t)b * p.max_blocks + t / p.bs];
-      if (id < 0 || id >= p.num_blocks) {
-        flag_error(PKV_DEVERR_BLOCK_ID);
-      } else {
-        dst = id;
-        row = t % p.bs;
-        const int c = p.cow_src != nullptr ? p.cow_src[b] : -1;
-        if (c >= p.num_blocks) flag_error(PKV_DEVERR_COPY);
-        else if (c >= 0 && c != id) src = c;
-      }
-    }
-    s_dst[threadIdx.x] = dst;
-    s_src[threadIdx.x] = src;
-    s_row[threadIdx.x] = row;
-  }
-}
-
-// Phase 2 (every thread, after that barrier): the copies and the new rows.
-template <typename T, int D>
-__device__ __forceinline__ void group_append_write(const DecodeParams& p, int lo, int members,
-                                                   int kvh, const int* s_dst, const int* s_src,
-                                                   const int* s_row) {
+// leave out).  The result equals copy_blocks then paged_kv_write.
+// Member i's blocks come from the warp's per-member words in shared memory: its
+// length (len), copy-on-write source (src, < 0: none) and row of the new token;
+// dst[i] is the block the new token goes to (< 0: nothing to write), filed by
+// resolve(), which runs once, after the first batch's reads are issued, so that
+// those reads and the block ids share one memory latency.  The threads read up to
+// kBatch elements each before writing any; the CTA's elements are taken in batches
+// of kBatch x blockDim.x.
+template <typename T, int D, class Resolve>
+__device__ __forceinline__ void group_append(const DecodeParams& p, int lo, int members, int kvh,
+                                             const int* len, const int* src, const int* row,
+                                             const int* dst, Resolve&& resolve) {
   constexpr int kVec = D * (int)sizeof(T) / 16;  // 16-byte vectors per head row
+  constexpr int kBatch = 8;
   const size_t row_vec = (size_t)p.Hkv * kVec;    // per token row (all heads)
   uint4* kc = reinterpret_cast<uint4*>(p.k_cache_w);
   uint4* vc = reinterpret_cast<uint4*>(p.v_cache_w);
   const uint4* kn = reinterpret_cast<const uint4*>(p.k_new);
   const uint4* vn = reinterpret_cast<const uint4*>(p.v_new);
   const int per = (p.bs + 1) * kVec;  // per member: the block's rows, then the new row
-  for (int x = threadIdx.x; x < members * per; x += blockDim.x) {
-    const int i = x / per, r = (x % per) / kVec, c = x % kVec;
-    const int dst = s_dst[i];
-    if (dst < 0) continue;
-    if (r == p.bs) {
-      const size_t d_o = ((size_t)dst * p.bs + s_row[i]) * row_vec + (size_t)kvh * kVec + c;
-      const size_t so = ((size_t)(lo + i) * p.Hkv + kvh) * kVec + c;
-      kc[d_o] = kn[so];
-      vc[d_o] = vn[so];
-    } else if (s_src[i] >= 0 && r != s_row[i]) {
-      const size_t so = ((size_t)s_src[i] * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
-      const size_t d_o = ((size_t)dst * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
-      kc[d_o] = kc[so];
-      vc[d_o] = vc[so];
+  const int total = members * per;
+  bool resolved = false;
+  for (int base = 0; base < total; base += kBatch * (int)blockDim.x) {
+    uint4 ka[kBatch], va[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int x = base + j * (int)blockDim.x + (int)threadIdx.x;
+      if (x >= total) break;
+      const int i = x / per, r = (x % per) / kVec, c = x % kVec;
+      if (len[i] <= 0) continue;
+      if (r == p.bs) {
+        const size_t so = ((size_t)(lo + i) * p.Hkv + kvh) * kVec + c;
+        ka[j] = kn[so];
+        va[j] = vn[so];
+      } else if (src[i] >= 0 && r != row[i]) {
+        const size_t so = ((size_t)src[i] * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
+        ka[j] = kc[so];
+        va[j] = vc[so];
+      }
+    }
+    if (!resolved) {
+      resolve();
+      resolved = true;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int x = base + j * (int)blockDim.x + (int)threadIdx.x;
+      if (x >= total) break;
+      const int i = x / per, r = (x % per) / kVec, c = x % kVec;
+      const int d = dst[i];
+      if (len[i] <= 0 || d < 0) continue;
+      if (r == p.bs) {
+        const size_t d_o = ((size_t)d * p.bs + row[i]) * row_vec + (size_t)kvh * kVec + c;
+        kc[d_o] = ka[j];
+        vc[d_o] = va[j];
+      } else if (src[i] >= 0 && src[i] != d && r != row[i]) {
+        const size_t d_o = ((size_t)d * p.bs + r) * row_vec + (size_t)kvh * kVec + c;
+        kc[d_o] = ka[j];
+        vc[d_o] = va[j];
+      }
     }
   }
+  if (!resolved) resolve();
   fence_proxy_async_global();
 }
 
@@ -417,20 +424,40 @@ struct GroupSmem {
   static constexpr size_t kBytes = 1024 /*alignment slack*/ + (size_t)W * kSlot + W * C::kStages * 8;
 };
 
+// The set-up takes two memory latencies before the stream runs: the first round
+// of loads (members' lengths, copy-on-write sources, the block ids of each warp's
+// first prefix stages) is issued before any stage load, so that it does not queue
+// behind them; each warp derives the prefix and the members' stage offsets from it
+// on its own (no CTA barrier) and starts its first prefix stages.  The second round
+// (ids of own-token stages, the members' table check, the fused step's blocks and
+// copy reads) runs while those stages are in flight.
+// app_bar completes once every thread has made its share of the fused step's
+// writes; only the loads of own-token stages wait for it.
 template <class C, int D, int W>
-__device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kvh, uint8_t* smem,
-                                            const CUtensorMap& tmK, const CUtensorMap& tmV) {
+__device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, int off_hi,
+                                            int plen_req, int kvh, uint8_t* smem,
+                                            uint64_t* app_bar, const CUtensorMap& tmK,
+                                            const CUtensorMap& tmV) {
   using T = __nv_bfloat16;
   constexpr int kRing = GroupSmem<C, D, W>::kSlot;  // stride of the warps' slots
   constexpr int kMaxMembers = 16;
   static_assert(C::GP == 16, "group pieces use the 16-row consumer");
-  __shared__ int s_len[kMaxMembers], s_cum[kMaxMembers + 1];
+  // Each warp's own copy of the members' words: length, first stage (s_cum[i], with
+  // s_cum[members] the CTA's stage count), copy-on-write source, new-token row and
+  // block.
+  __shared__ int s_len[W][kMaxMembers], s_cum[W][kMaxMembers + 1];
+  __shared__ int s_src[W][kMaxMembers], s_row[W][kMaxMembers], s_dst[W][kMaxMembers];
+  // Stage meta words (valid tokens | member << 5 | every-row flag << 10), filed by
+  // lane 0 beside the stage's slot when it loads the stage.
+  __shared__ int s_meta[W][C::kStages];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * kRing);
   const DecodeParams& p = s.d;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
   T* out = reinterpret_cast<T*>(p.out);
-  const int lo = group_off(s, g), hi = max(lo, group_off(s, g + 1));
+  // Group offsets are caller data: clamped into [0, B], so that no value of theirs
+  // leads outside the batch.
+  const int lo = min(max(off_lo, 0), p.B), hi = max(lo, min(max(off_hi, 0), p.B));
   int members = hi - lo;
   if (members <= 0) return;
   const int mc = min(s.mc, kMaxMembers);
@@ -438,7 +465,6 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     if (threadIdx.x == 0) flag_error(PKV_DEVERR_PREFIX);
     members = mc;
   }
-  const int plen = group_prefix(s, g, lo, hi);  // whole blocks
   uint8_t* ring = smem + warp * kRing;
   uint64_t* wbar = bars + warp * C::kStages;
   if (lane == 0) {
@@ -450,107 +476,85 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
   }
   __syncwarp();
   const uint64_t pol = l2_policy_evict_first();
-  // Stage meta words (valid tokens | member << 5 | every-row flag << 10), filed by
-  // lane 0 beside the stage's slot when it loads the stage.
-  __shared__ int s_meta[W][C::kStages];
-  // This warp's first stages (warp, warp + W, ...) that lie in the shared prefix
-  // need nothing but the first member's table row: their loads start before the
-  // fused step's writes and the set-up below (those writes never touch a prefix
-  // block, which ends before every member's newest token and on a block boundary).
-  int n_early = 0;
-  {
-    const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
-    const int n_pre0 = plen / kStageTokens;
-#pragma unroll
-    for (int kk = 0; kk < C::kStages; ++kk) {
-      const int k = warp + W * kk;
-      if (k >= n_pre0) break;
-      if (lane == 0) {
-        const int t0 = k * kStageTokens;
-        const int id = r0[t0 / p.bs];
-        int row = p.num_blocks * p.bs;  // past the pool: TMA fills zeros
-        if (id < 0 || id >= p.num_blocks) flag_error(PKV_DEVERR_BLOCK_ID);
-        else row = id * p.bs + t0 % p.bs;
-        s_meta[warp][kk] = kStageTokens | (1 << 10);
-        mbar_arrive_expect_tx(&wbar[kk], C::kStageBytes);
-        C::load_stage(ring + kk * C::kStageBytes, &tmK, &tmV, &wbar[kk], kvh, row, pol);
-      }
-      ++n_early;
-    }
-  }
-  // Set-up: each member's stage count (s_cum) and, for a fused step, the blocks its
-  // new token goes to; then the fused step's writes (every member's new token after
-  // any copy-on-write of its block) land before any stage of own tokens is loaded.
   const bool fused = p.k_new != nullptr;
-  __shared__ int s_adst[kMaxMembers], s_asrc[kMaxMembers], s_arow[kMaxMembers];
-  if (fused) group_append_resolve(p, lo, members, s_adst, s_asrc, s_arow);
-  if (threadIdx.x == blockDim.x - 1) {
-    int cum = plen / kStageTokens;
-    s_cum[0] = cum;
-    for (int i = 0; i < members; ++i) {
-      const int L = shared_len(p, lo + i);
-      s_len[i] = L;
-      cum += L > plen ? (L - plen + kStageTokens - 1) / kStageTokens : 0;
-      s_cum[i + 1] = cum;
-    }
+  const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
+
+  // Round 1.  Lane i: member i's length and copy-on-write source.  Every lane: the
+  // block id of the warp's stage warp + W * lane, read as a prefix stage when the
+  // caller's prefix reaches it (used only if the actual prefix does too).
+  const int cap_pre = min(max(plen_req, 0), p.max_blocks * p.bs) / kStageTokens;
+  const int kw = warp + W * lane;
+  int win0p = kw < cap_pre ? r0[kw * kStageTokens / p.bs] : -1;
+  int Li = 0, ci = -1;
+  if (lane < members) {
+    Li = shared_len(p, lo + lane);
+    if (fused && p.cow_src != nullptr) ci = p.cow_src[lo + lane];
   }
-  __syncthreads();
-  if (fused) group_append_write<T, D>(p, lo, members, kvh, s_adst, s_asrc, s_arow);
-  {  // every member must hold the same physical blocks for the prefix
-    const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
-    const int nj = plen > 0 ? (plen - 1) / p.bs + 1 : 0;
-    for (int x = threadIdx.x; x < nj * members; x += blockDim.x) {
-      const int j = x % nj, b = lo + x / nj;
-      if (p.block_tables[(size_t)b * p.max_blocks + j] != r0[j]) flag_error(PKV_DEVERR_PREFIX);
-    }
+  // The prefix actually shared: short of every member's newest token (so no block
+  // of it is one the fused step writes) and whole blocks.
+  const int min_last = __reduce_min_sync(kFull, lane < members ? Li - 1 : 0x7fffffff);
+  const int plen = max(0, min(plen_req, min_last)) / p.bs * p.bs;
+  const int n_pre = plen / kStageTokens;
+  int cum = (lane < members && Li > plen) ? (Li - plen + kStageTokens - 1) / kStageTokens : 0;
+#pragma unroll
+  for (int d = 1; d < 32; d *= 2) {
+    const int y = __shfl_up_sync(kFull, cum, d);
+    if (lane >= d) cum += y;
   }
-  if (fused) __syncthreads();
-  const int n_pre = s_cum[0], n_all = s_cum[members];
-  // Stage k of the CTA: the member i whose table row it reads, its first token
-  // and its valid tokens; true when every member's rows score it (a prefix stage,
-  // or any stage of a one-member group), else only member i's rows do.
-  auto stage_of = [&](int k, int& i, int& t0, int& nv) -> bool {
-    i = 0;
-    if (k < n_pre) {
-      t0 = k * kStageTokens;
-      nv = kStageTokens;
-      return true;
-    }
-    while (k >= s_cum[i + 1]) ++i;
-    t0 = plen + (k - s_cum[i]) * kStageTokens;
-    nv = min(kStageTokens, s_len[i] - t0);
-    return members == 1;
-  };
-  // This warp takes the CTA's stages warp, warp + W, ...
+  if (lane < members) {
+    s_len[warp][lane] = Li;
+    s_cum[warp][lane + 1] = n_pre + cum;
+    s_src[warp][lane] = ci >= 0 && ci < p.num_blocks ? ci : -1;
+    s_row[warp][lane] = Li > 0 ? (Li - 1) % p.bs : 0;
+  }
+  if (lane == 0) s_cum[warp][0] = n_pre;
+  const int n_all = n_pre + __shfl_sync(kFull, cum, 31);
+  __syncwarp();
+
+  // This warp takes the CTA's stages warp, warp + W, ...; its stages win_base ..
+  // win_base + 63 have their block ids resolved ahead, one per lane of two windows.
+  // Window 0 holds prefix ids (win0p, round 1) and own-token ids (win0t, round 2)
+  // apart, so that issuing a prefix stage never waits for a round-2 load.
   const int first = warp, stride = W;
   const int n_w = n_all > first ? (n_all - first + stride - 1) / stride : 0;
-  // The warp's stages win_base .. win_base + 63 are resolved ahead, one per lane
-  // of two windows: the TMA row of the stage's 16 tokens (past the pool, so
-  // that TMA fills zeros, for a block id out of range) and its meta word.
-  auto stage_info = [&](int kk, int& meta) -> int {
-    int i, t0, nv;
-    const bool all_rows = stage_of(first + stride * kk, i, t0, nv);
-    meta = nv | (i << 5) | (all_rows ? 1 << 10 : 0);
-    const int id = p.block_tables[(size_t)(lo + i) * p.max_blocks + t0 / p.bs];
-    if (id < 0 || id >= p.num_blocks) {
-      flag_error(PKV_DEVERR_BLOCK_ID);
-      return p.num_blocks * p.bs;
-    }
-    return id * p.bs + t0 % p.bs;
+  auto stage_id = [&](int k) -> int {  // block id of the CTA's stage k, or -1
+    if (k >= n_all) return -1;
+    if (k < n_pre) return r0[k * kStageTokens / p.bs];
+    int i = 0;
+    while (k >= s_cum[warp][i + 1]) ++i;
+    const int t0 = plen + (k - s_cum[warp][i]) * kStageTokens;
+    return p.block_tables[(size_t)(lo + i) * p.max_blocks + t0 / p.bs];
   };
-  int win_base = 0, wm0 = 0, wm1 = 0;
-  int win0 = lane < n_w ? stage_info(lane, wm0) : 0;
-  int win1 = 32 + lane < n_w ? stage_info(32 + lane, wm1) : 0;
+  int win_base = 0, win0t = -1, win1 = -1;
+  bool app_seen = !fused;  // lane 0: the fused step's writes are known to have landed
   auto issue = [&](int kk) {
     if (kk - win_base >= 32) {
-      win0 = win1;
-      wm0 = wm1;
+      win0p = win1;
+      win0t = win1;
       win_base += 32;
-      win1 = win_base + 32 + lane < n_w ? stage_info(win_base + 32 + lane, wm1) : 0;
+      win1 = stage_id(first + stride * (win_base + 32 + lane));
     }
-    const int row = __shfl_sync(kFull, win0, kk - win_base);  // kk - win_base < 32 here
-    const int meta = __shfl_sync(kFull, wm0, kk - win_base);
+    const int k = first + stride * kk;
+    const int id = k < n_pre ? __shfl_sync(kFull, win0p, kk - win_base)
+                             : __shfl_sync(kFull, win0t, kk - win_base);
     if (lane == 0) {
+      if (k >= n_pre && !app_seen) {
+        if (!mbar_wait_bounded(app_bar, 0)) flag_error(PKV_DEVERR_TIMEOUT);
+        app_seen = true;
+      }
+      int t0, meta;
+      if (k < n_pre) {
+        t0 = k * kStageTokens;
+        meta = kStageTokens | (1 << 10);  // every member's rows score it
+      } else {
+        int i = 0;
+        while (k >= s_cum[warp][i + 1]) ++i;
+        t0 = plen + (k - s_cum[warp][i]) * kStageTokens;
+        meta = min(kStageTokens, s_len[warp][i] - t0) | (i << 5) | (members == 1 ? 1 << 10 : 0);
+      }
+      int row = p.num_blocks * p.bs;  // past the pool: TMA fills zeros
+      if (id < 0 || id >= p.num_blocks) flag_error(PKV_DEVERR_BLOCK_ID);
+      else row = id * p.bs + t0 % p.bs;
       const int st = kk % C::kStages;
       s_meta[warp][st] = meta;
       mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
@@ -558,8 +562,58 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int g, int kv
     }
     __syncwarp();  // the meta word is seen by every lane before the stage is consumed
   };
+  // The first stages that lie in the prefix load now: a prefix block is never one
+  // that the fused step writes.
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
-  for (int kk = n_early; kk < n_pro; ++kk) issue(kk);  // the early ones are in flight
+  int n_early = 0;
+  while (n_early < n_pro && first + stride * n_early < n_pre) issue(n_early++);
+
+  // Round 2, while those stages are in flight.
+  win0t = kw >= n_pre ? stage_id(kw) : -1;
+  win1 = stage_id(first + stride * (32 + lane));
+  // Every member must hold the same physical blocks for the prefix: entry j of
+  // member i (i >= 1) against member 0's.  Two entries a thread are read now and
+  // compared after the step's writes; the rest (long prefixes) after that.
+  const int nj = plen / p.bs, n_chk = (members - 1) * nj;
+  int chk_a[2] = {0, 0}, chk_b[2] = {0, 0};
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int x = (int)threadIdx.x + j * (int)blockDim.x;
+    if (x < n_chk) {
+      chk_a[j] = p.block_tables[(size_t)(lo + 1 + x / nj) * p.max_blocks + x % nj];
+      chk_b[j] = r0[x % nj];
+    }
+  }
+  if (fused) {
+    // Lane i: the block member i's new token goes to, read in the same latency as
+    // the first copy reads and filed before any write.
+    int id = -1;
+    if (lane < members && Li > 0)
+      id = p.block_tables[(size_t)(lo + lane) * p.max_blocks + (Li - 1) / p.bs];
+    auto resolve = [&] {
+      if (lane < members) {
+        int d = -1;
+        if (Li > 0) {
+          if (id < 0 || id >= p.num_blocks) {
+            if (warp == 0) flag_error(PKV_DEVERR_BLOCK_ID);
+          } else {
+            d = id;
+            if (ci >= p.num_blocks && warp == 0) flag_error(PKV_DEVERR_COPY);
+          }
+        }
+        s_dst[warp][lane] = d;
+      }
+      __syncwarp();
+    };
+    group_append<T, D>(p, lo, members, kvh, s_len[warp], s_src[warp], s_row[warp], s_dst[warp],
+                       resolve);
+    mbar_arrive(app_bar);  // release: this thread's writes, fenced for the TMA reads
+  }
+  bool chk_ok = chk_a[0] == chk_b[0] && chk_a[1] == chk_b[1];
+  for (int x = (int)threadIdx.x + 2 * (int)blockDim.x; x < n_chk; x += blockDim.x)
+    chk_ok &= p.block_tables[(size_t)(lo + 1 + x / nj) * p.max_blocks + x % nj] == r0[x % nj];
+  if (!chk_ok) flag_error(PKV_DEVERR_PREFIX);
+  while (n_early < n_pro) issue(n_early++);
 
   C c;
   c.init_gather(p, lo, members, kvh, lane);
@@ -645,13 +699,24 @@ __global__ void __launch_bounds__(W * 32, D <= 128 ? 2 : 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  if (cta_timed_out()) return;
-  if (blockIdx.x == 0 && threadIdx.x == 0) {  // the groups must tile the batch in order
-    bool ok = s.group_offsets[0] == 0 && s.group_offsets[s.n_groups] == s.d.B;
-    for (int g = 0; g < s.n_groups && ok; ++g) ok = s.group_offsets[g] <= s.group_offsets[g + 1];
+  const int g = (int)blockIdx.x / s.d.Hkv, kvh = (int)blockIdx.x % s.d.Hkv;
+  // The group's bounds and asked-for prefix are read before the timeout check, so
+  // that the two latencies overlap.
+  const int off_lo = s.group_offsets[g], off_hi = s.group_offsets[g + 1];
+  const int plen_req = s.prefix_lens[g];
+  __shared__ uint64_t s_app;  // the fused step's writes: one arrival per thread
+  if (threadIdx.x == 0) {
+    mbar_init(&s_app, W * 32);
+    fence_mbar_init();
+  }
+  if (cta_timed_out()) return;  // its barrier also publishes the initialised s_app
+  if (kvh == 0 && threadIdx.x == 0) {  // the groups must tile the batch in order
+    bool ok = off_lo <= off_hi;
+    if (g == 0) ok = ok && off_lo == 0;
+    if (g == s.n_groups - 1) ok = ok && off_hi == s.d.B;
     if (!ok) flag_error(PKV_DEVERR_PREFIX);
   }
-  group_piece<C, D, W>(s, (int)blockIdx.x / s.d.Hkv, (int)blockIdx.x % s.d.Hkv, smem, tmK, tmV);
+  group_piece<C, D, W>(s, off_lo, off_hi, plen_req, kvh, smem, &s_app, tmK, tmV);
 }
 
 template <class C2, class C1, int D>
