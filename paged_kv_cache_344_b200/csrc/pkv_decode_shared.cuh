@@ -490,6 +490,13 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     Li = shared_len(p, lo + lane);
     if (fused && p.cow_src != nullptr) ci = p.cow_src[lo + lane];
   }
+  {  // the members' q rows of this KV head (read at the end of the set-up) into L2
+    const int lines = G * D * (int)sizeof(T) / 128;  // per member, contiguous
+    const uint8_t* q0 = reinterpret_cast<const uint8_t*>(p.q) +
+                        ((size_t)lo * p.Hq + (size_t)kvh * G) * D * sizeof(T);
+    for (int x = lane; x < members * lines; x += 32)
+      prefetch_l2_line(q0 + (size_t)(x / lines) * p.Hq * D * sizeof(T) + (size_t)(x % lines) * 128);
+  }
   // The prefix actually shared: short of every member's newest token (so no block
   // of it is one the fused step writes) and whole blocks.
   const int min_last = __reduce_min_sync(kFull, lane < members ? Li - 1 : 0x7fffffff);
@@ -562,13 +569,17 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     }
     __syncwarp();  // the meta word is seen by every lane before the stage is consumed
   };
-  // The first stages that lie in the prefix load now: a prefix block is never one
-  // that the fused step writes.
+  // The first stages that lie in the prefix: a prefix block is never one that the
+  // fused step writes.  They load after round 2 is issued, so that round 2 does not
+  // queue behind every warp's first stages.
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
   int n_early = 0;
-  while (n_early < n_pro && first + stride * n_early < n_pre) issue(n_early++);
+  auto first_stages = [&] {
+    while (n_early < n_pro && first + stride * n_early < n_pre) issue(n_early++);
+  };
 
-  // Round 2, while those stages are in flight.
+  // Round 2: ids of the own-token stages, the members' table check, and for a fused
+  // step each member's new-token block and the first batch of its copy reads.
   win0t = kw >= n_pre ? stage_id(kw) : -1;
   win1 = stage_id(first + stride * (32 + lane));
   // Every member must hold the same physical blocks for the prefix: entry j of
@@ -585,12 +596,12 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     }
   }
   if (fused) {
-    // Lane i: the block member i's new token goes to, read in the same latency as
-    // the first copy reads and filed before any write.
+    // Lane i: the block member i's new token goes to, filed before any write.
     int id = -1;
     if (lane < members && Li > 0)
       id = p.block_tables[(size_t)(lo + lane) * p.max_blocks + (Li - 1) / p.bs];
     auto resolve = [&] {
+      first_stages();
       if (lane < members) {
         int d = -1;
         if (Li > 0) {
@@ -608,6 +619,8 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     group_append<T, D>(p, lo, members, kvh, s_len[warp], s_src[warp], s_row[warp], s_dst[warp],
                        resolve);
     mbar_arrive(app_bar);  // release: this thread's writes, fenced for the TMA reads
+  } else {
+    first_stages();
   }
   bool chk_ok = chk_a[0] == chk_b[0] && chk_a[1] == chk_b[1];
   for (int x = (int)threadIdx.x + 2 * (int)blockDim.x; x < n_chk; x += blockDim.x)
