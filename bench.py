@@ -83,6 +83,18 @@ def kernel_source_sha(kind: str = "decode") -> str:
     return h.hexdigest()[:16]
 
 
+# A device-side wait enqueued right before each timed region.  While it runs, the host
+# enqueues the first timed launches, so that host start-up work (the clock sampler's
+# first NVML calls, the first launches' argument marshalling) never shows up inside the
+# region as GPU idle time.  It lies outside the timed events.
+PRIME_CYCLES = 4_000_000  # about 2 ms at 1965 MHz
+
+
+def prime_queue():
+    import torch
+    torch.cuda._sleep(PRIME_CYCLES)
+
+
 def recorded_traffic(config: str, partition: int, kind: str = "decode"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel sources (and, for decode, the same partition length); else None."""
@@ -138,6 +150,10 @@ class ClockSampler:
             self.nv = pynvml
             self.h = self._handle(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            # The first queries of a process are slow and can hold up the next kernel
+            # launch; take them here, before any timed region starts.
+            pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons()
             self.ok = True
         except Exception as e:  # no NVML: report clocks as unavailable
             self.err = str(e)
@@ -165,12 +181,15 @@ class ClockSampler:
                 self.reasons |= int(self._reasons())
             except Exception:
                 pass
+            self._first.set()
             time.sleep(self.period)
 
     def __enter__(self):
         if self.ok:
+            self._first = threading.Event()
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
+            self._first.wait(1.0)  # the thread's start-up lies before the timed region
         return self
 
     def __exit__(self, *a):
@@ -360,8 +379,10 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
 
     for _ in range(warmup):
         step(d_in)
+    prime_queue()  # its first launch loads the kernel; not inside a timed region
     if flush:
         scratch.fill_(1)
+        scratch.add_(1)  # likewise the flush's kernel, which runs before every timed step
     barrier()
 
     def timed_region():
@@ -369,11 +390,18 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
                   for _ in range(steps)]
         ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(steps)]
-        barrier()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
+        # A CUDA event is created at its first record; the first creations of a process
+        # are slow.  Record every event once here, so that none is created between a
+        # step's launch and its end event inside the region.
+        for a, b in ev_dec + ev_step + [(t_start, t_end)]:
+            a.record(stream)
+            b.record(stream)
+        barrier()
         with ClockSampler(local_rank) as clocks:
             torch.cuda.nvtx.range_push("timed_region")
+            prime_queue()
             t_start.record(stream)
             for i in range(steps):
                 if flush:
@@ -494,8 +522,10 @@ def run_e2e(step, d_in, out, has_cow, stream, step_bytes, wl, world, dev_name, s
             d2h_(i)
 
     e2e_run(max(3, warmup // 4))
-    barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)  # created now, not inside the region
+    e1.record(stream)
+    barrier()
     e2e_steps = max(10, steps // 4)
     e0.record(copy_s)
     e2e_run(e2e_steps)
@@ -583,9 +613,13 @@ def run_prefill(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         step()
-    torch.cuda.synchronize()
+    prime_queue()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)  # created now, not inside the region
+    e1.record(stream)
+    torch.cuda.synchronize()
     with ClockSampler(local_rank) as clocks:
+        prime_queue()
         e0.record(stream)
         for _ in range(args.steps):
             step()
@@ -699,6 +733,7 @@ def run_paging(args, local_rank):
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
+        prime_queue()
         for a, b in ev:
             if flush:
                 scratch.add_(1)
