@@ -265,13 +265,19 @@ def custom(name, dtype, B, Hq, Hkv, D, bs, seq_lens_pre, seed, pool_factor=1.25,
 def grouped(name, dtype, Hq, Hkv, D, bs, group_sizes, shared_tokens, tails, seed,
             pool_factor=1.25):
     """Groups of consecutive sequences that share a prefix of ``shared_tokens[g]`` tokens
-    (same physical blocks), each member followed by ``tails[b]`` tokens of its own."""
+    (same physical blocks), each member followed by ``tails[b]`` tokens of its own.  A prefix
+    that ends inside a block is a fork: its members hold no tokens of their own yet, they
+    share the partly filled block, and the step copies it on write for all but its last
+    holder."""
     rng = np.random.default_rng(seed)
     groups = np.repeat(np.arange(len(group_sizes)), group_sizes)
     shared = np.asarray(shared_tokens, dtype=np.int64)
-    # Members write their own tokens after the prefix, so it must end on a block boundary.
-    assert np.all(shared % bs == 0), "shared prefixes must be whole blocks"
-    L = shared[groups] + np.asarray(tails, dtype=np.int64)
+    own = np.asarray(tails, dtype=np.int64)
+    # Members write their own tokens after the prefix, so a prefix that ends inside a
+    # block leaves them none.
+    fork = (shared % bs != 0)[groups]
+    assert np.all(own[fork] == 0), "a prefix ending inside a block is a fork: no own tokens"
+    L = shared[groups] + own
     return _build(name, dtype, len(groups), Hq, Hkv, D, bs, L, seed, rng,
                   pool_factor=pool_factor, groups=groups, shared_tokens=shared)
 
