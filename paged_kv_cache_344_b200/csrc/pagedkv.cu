@@ -517,6 +517,9 @@ int decode_impl(void* out, const void* q, const void* k_cache, const void* v_cac
   p.max_parts = shape.max_parts;
   p.num_blocks = (int)num_blocks;
   p.scale_log2 = scale * 1.4426950408889634f;
+  // A few sequences cut into long partitions: CTAs in length order, so that the
+  // shortest start last (measured on the long-context workload).
+  p.sorted = !shape.balanced && B <= pkv::kSortedMaxB && shape.P >= 2048 ? 1 : 0;
   if (fused) {
     p.k_new = step.k_new;
     p.v_new = step.v_new;

@@ -79,6 +79,9 @@ struct DecodeParams {
   void* k_cache_w;       // the caches, written by the fused step
   void* v_cache_w;
   const int32_t* cow_src;  // [B] or null: block copied into the new token's block first
+  // Nonzero: CTAs take their (sequence, partition, KV head) in length order
+  // (sorted_item) instead of from their grid coordinates.
+  int sorted;
 };
 
 template <typename T>
@@ -751,6 +754,81 @@ enum : int {
                       // no block table at all; the control for the paging overhead
 };
 
+// Length order, for a few long sequences (B <= kSortedMaxB).  CTAs start in
+// the order of their linear block index, and one of them lasts a whole partition,
+// so the ones that start last set the end of the launch.  CTA number i therefore
+// takes the i-th item of this order: every full partition first (by sequence,
+// partition, KV head), then each sequence's last partition from the longest to the
+// shortest (an empty sequence counts as a last partition of 0 tokens), so that the
+// SMs run out of work together.  Each CTA derives the order from the lengths; it
+// returns false when i lies past the last item.
+constexpr int kSortedMaxB = 64;
+
+__device__ __forceinline__ bool sorted_item(const DecodeParams& p, int& b, int& part, int& kvh) {
+  __shared__ int s_full[kSortedMaxB + 1];  // full partitions of the sequences before b
+  __shared__ int s_last[kSortedMaxB];      // tokens of each sequence's last partition
+  __shared__ int s_sel;
+  const int B = p.B, P = p.part_tokens, Hkv = p.Hkv;
+  const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
+  const int t = threadIdx.x, lane = t % 32;
+  const long long i =
+      blockIdx.x + (long long)gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
+  if (t < 32) {  // lane l: sequences 2l and 2l + 1
+    int c[2] = {0, 0};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int x = 2 * lane + h;
+      if (x < B) {
+        int L = p.seq_lens[x];
+        L = L < 0 ? 0 : min(L, Lcap);
+        const int n = (L + P - 1) / P;
+        c[h] = max(n - 1, 0);
+        s_last[x] = L - c[h] * P;
+      }
+    }
+    int inc = c[0] + c[1];  // inclusive scan of the pairs over the lanes
+#pragma unroll
+    for (int d = 1; d < 32; d *= 2) {
+      const int y = __shfl_up_sync(kFull, inc, d);
+      if (lane >= d) inc += y;
+    }
+    const int before = inc - c[0] - c[1];
+    if (2 * lane < B) s_full[2 * lane + 1] = before + c[0];
+    if (2 * lane + 1 < B) s_full[2 * lane + 2] = before + c[0] + c[1];
+    if (lane == 0) s_full[0] = 0;
+  }
+  __syncthreads();
+  const long long f = i / Hkv;
+  kvh = (int)(i % Hkv);
+  const int F = s_full[B];
+  if (f < F) {
+    int lo = 0, hi = B;  // s_full[lo] <= f < s_full[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (s_full[mid] <= f) lo = mid;
+      else hi = mid;
+    }
+    b = lo;
+    part = (int)(f - s_full[lo]);
+    return true;
+  }
+  const long long j = f - F;
+  if (j >= B) return false;
+  if (t < B) {
+    const int mine = s_last[t];
+    int rank = 0;
+    for (int x = 0; x < B; ++x) {
+      const int o = s_last[x];
+      rank += (o > mine) || (o == mine && x < t);
+    }
+    if (rank == j) s_sel = t;
+  }
+  __syncthreads();
+  b = s_sel;
+  part = s_full[b + 1] - s_full[b];  // its full partitions come before the last one
+  return true;
+}
+
 template <class C, typename T, int D, int LAYOUT = kLayoutPaged>
 __global__ void __launch_bounds__(kWarps * 32)
     paged_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
@@ -764,13 +842,14 @@ __global__ void __launch_bounds__(kWarps * 32)
   __shared__ float s_M[16], s_den[16];
   __shared__ int s_last;
 
-  const int kvh = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
+  int kvh = blockIdx.x, part = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int G = p.G;
   const int P = p.part_tokens;
 
   // After a pipeline timeout anywhere, later CTAs stop at once instead of waiting too.
   if (cta_timed_out()) return;
+  if (p.sorted && !sorted_item(p, b, part, kvh)) return;
   int L = p.seq_lens[b];
   const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
   if (L < 0 || L > Lcap) {
