@@ -405,6 +405,48 @@ __device__ __forceinline__ void group_append(const DecodeParams& p, int lo, int 
   fence_proxy_async_global();
 }
 
+// A member's last stage when the fused step writes through the stages (blocks of
+// 16 tokens, so the stage is the block): the new token's K and V rows go into row
+// r of the stage in shared memory, in the 128-byte-swizzled layout the TMA boxes
+// land in (16-byte chunk c of a row at position c ^ (row % 8) of its 64-dim
+// sub-tile).  Then the block goes out to its destination d from there: all of it
+// when it is a copy of block src (the stage was loaded from src), else row r
+// alone.  Nothing in this launch reads those bytes of the pool again.  Each
+// element of the pool is written once, as by copy_blocks then paged_kv_write.
+template <class C, typename T, int D>
+__device__ __forceinline__ void group_patch_stage(const DecodeParams& p, uint8_t* st,
+                                                  const uint4* nrow, int r, int d, int src,
+                                                  int kvh, int lane) {
+  constexpr int kRowChunks = D * (int)sizeof(T) / 16;  // 16-byte chunks of one head row
+  constexpr int kSub = kStageTokens * 128;             // one 64-dim sub-tile
+  cp_async_wait_all();  // this lane's copies of the new rows; the barrier shows all
+  __syncwarp();
+  auto at = [&](int kv, int row, int cc) -> uint4* {
+    return reinterpret_cast<uint4*>(st + kv * C::kTileBytes + (cc / 8) * kSub + row * 128 +
+                                    (((cc % 8) ^ (row & 7)) << 4));
+  };
+  for (int x = lane; x < 2 * kRowChunks; x += 32) *at(x / kRowChunks, r, x % kRowChunks) = nrow[x];
+  fence_proxy_async_smem();  // before the slot's next TMA fill
+  __syncwarp();
+  if (d < 0) return;
+  uint4* kc = reinterpret_cast<uint4*>(p.k_cache_w);
+  uint4* vc = reinterpret_cast<uint4*>(p.v_cache_w);
+  const size_t row_vec = (size_t)p.Hkv * kRowChunks;  // per token row (all heads)
+  const size_t head = (size_t)kvh * kRowChunks;
+  if (src >= 0 && src != d) {
+    for (int x = lane; x < 2 * kStageTokens * kRowChunks; x += 32) {
+      const int kv = x / (kStageTokens * kRowChunks), rem = x % (kStageTokens * kRowChunks);
+      const int row = rem / kRowChunks, cc = rem % kRowChunks;
+      (kv ? vc : kc)[((size_t)d * kStageTokens + row) * row_vec + head + cc] = *at(kv, row, cc);
+    }
+  } else {
+    for (int x = lane; x < 2 * kRowChunks; x += 32) {
+      const int kv = x / kRowChunks, cc = x % kRowChunks;
+      (kv ? vc : kc)[((size_t)d * kStageTokens + r) * row_vec + head + cc] = nrow[x];
+    }
+  }
+}
+
 // One CTA for a whole group and one KV head, when the group's members fit the
 // 16 query rows of one MMA (members <= 16 / G).  The CTA's stages are the
 // shared prefix's (scored for every member's rows) followed by each member's
@@ -447,9 +489,14 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
   // block.
   __shared__ int s_len[W][kMaxMembers], s_cum[W][kMaxMembers + 1];
   __shared__ int s_src[W][kMaxMembers], s_row[W][kMaxMembers], s_dst[W][kMaxMembers];
-  // Stage meta words (valid tokens | member << 5 | every-row flag << 10), filed by
-  // lane 0 beside the stage's slot when it loads the stage.
+  // Stage meta words (valid tokens | member << 5 | every-row flag << 10 | the
+  // member's last stage << 11), filed by lane 0 beside the stage's slot when it
+  // loads the stage.
   __shared__ int s_meta[W][C::kStages];
+  // With 16-token blocks the fused step's writes go through the stages: the new
+  // K and V rows of a member whose last stage a slot holds, copied in beside it.
+  constexpr int kNewChunks = 2 * D * (int)sizeof(T) / 16;
+  __shared__ uint4 s_new[W][C::kStages][kNewChunks];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + W * kRing);
   const DecodeParams& p = s.d;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -477,6 +524,10 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
   __syncwarp();
   const uint64_t pol = l2_policy_evict_first();
   const bool fused = p.k_new != nullptr;
+  // A block is one stage: a member's last stage is loaded from its copy-on-write
+  // source, the new row is put in place in shared memory, and the block is written
+  // out from there (no copy pass, no wait on one).
+  const bool patch = fused && p.bs == kStageTokens;
   const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
 
   // Round 1.  Lane i: member i's length and copy-on-write source.  Every lane: the
@@ -533,7 +584,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     return p.block_tables[(size_t)(lo + i) * p.max_blocks + t0 / p.bs];
   };
   int win_base = 0, win0t = -1, win1 = -1;
-  bool app_seen = !fused;  // lane 0: the fused step's writes are known to have landed
+  bool app_seen = !fused || patch;  // lane 0: the fused step's writes are known to have landed
   auto issue = [&](int kk) {
     if (kk - win_base >= 32) {
       win0p = win1;
@@ -558,16 +609,34 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
         while (k >= s_cum[warp][i + 1]) ++i;
         t0 = plen + (k - s_cum[warp][i]) * kStageTokens;
         meta = min(kStageTokens, s_len[warp][i] - t0) | (i << 5) | (members == 1 ? 1 << 10 : 0);
+        if (patch && k == s_cum[warp][i + 1] - 1) meta |= 1 << 11;
       }
       int row = p.num_blocks * p.bs;  // past the pool: TMA fills zeros
-      if (id < 0 || id >= p.num_blocks) flag_error(PKV_DEVERR_BLOCK_ID);
-      else row = id * p.bs + t0 % p.bs;
+      if (id < 0 || id >= p.num_blocks) {
+        flag_error(PKV_DEVERR_BLOCK_ID);
+      } else {
+        row = id * p.bs + t0 % p.bs;
+        const int src = (meta >> 11) ? s_src[warp][(meta >> 5) & 31] : -1;
+        if (src >= 0 && src != id) row = src * p.bs;  // the block it is a copy of
+      }
       const int st = kk % C::kStages;
       s_meta[warp][st] = meta;
       mbar_arrive_expect_tx(&wbar[st], C::kStageBytes);
       C::load_stage(ring + st * C::kStageBytes, &tmK, &tmV, &wbar[st], kvh, row, pol);
     }
     __syncwarp();  // the meta word is seen by every lane before the stage is consumed
+    const int st = kk % C::kStages;
+    const int m = s_meta[warp][st];
+    if (m >> 11) {  // the member's new K and V rows, beside the slot
+      const int i = (m >> 5) & 31;
+      const uint4* kn = reinterpret_cast<const uint4*>(p.k_new);
+      const uint4* vn = reinterpret_cast<const uint4*>(p.v_new);
+      const size_t base = ((size_t)(lo + i) * p.Hkv + kvh) * (kNewChunks / 2);
+      for (int x = lane; x < kNewChunks; x += 32)
+        cp_async16(&s_new[warp][st][x],
+                   x < kNewChunks / 2 ? kn + base + x : vn + base + x - kNewChunks / 2);
+      cp_async_commit();
+    }
   };
   // The first stages that lie in the prefix: a prefix block is never one that the
   // fused step writes.  They load after round 2 is issued, so that round 2 does not
@@ -616,9 +685,13 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
       }
       __syncwarp();
     };
-    group_append<T, D>(p, lo, members, kvh, s_len[warp], s_src[warp], s_row[warp], s_dst[warp],
-                       resolve);
-    mbar_arrive(app_bar);  // release: this thread's writes, fenced for the TMA reads
+    if (patch) {
+      resolve();
+    } else {
+      group_append<T, D>(p, lo, members, kvh, s_len[warp], s_src[warp], s_row[warp],
+                         s_dst[warp], resolve);
+      mbar_arrive(app_bar);  // release: this thread's writes, fenced for the TMA reads
+    }
   } else {
     first_stages();
   }
@@ -641,10 +714,14 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     }
     const int meta = s_meta[warp][st];
     const int nv = meta & 31, r0 = ((meta >> 5) & 31) * G;
+    if (meta >> 11)
+      group_patch_stage<C, T, D>(p, ring + st * C::kStageBytes, s_new[warp][st], nv - 1,
+                                 s_dst[warp][(meta >> 5) & 31], s_src[warp][(meta >> 5) & 31],
+                                 kvh, lane);
     auto refill = [&] {
       if (kk + C::kStages < n_w) issue(kk + C::kStages);
     };
-    if (meta >> 10)  // every member's rows score it
+    if ((meta >> 10) & 1)  // every member's rows score it
       c.consume(ring + st * C::kStageBytes, nv, lane, refill);
     else
       c.consume_rows(ring + st * C::kStageBytes, nv, lane, r0, r0 + G, refill);
