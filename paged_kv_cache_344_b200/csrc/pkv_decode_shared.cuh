@@ -466,11 +466,11 @@ struct GroupSmem {
   static constexpr size_t kBytes = 1024 /*alignment slack*/ + (size_t)W * kSlot + W * C::kStages * 8;
 };
 
-// The set-up takes two memory latencies before the stream runs: the first round
+// The set-up takes two memory latencies before the stream runs: the first batch
 // of loads (members' lengths, copy-on-write sources, the block ids of each warp's
 // first prefix stages) is issued before any stage load, so that it does not queue
 // behind them; each warp derives the prefix and the members' stage offsets from it
-// on its own (no CTA barrier) and starts its first prefix stages.  The second round
+// on its own (no CTA barrier) and starts its first prefix stages.  The second batch
 // (ids of own-token stages, the members' table check, the fused step's blocks and
 // copy reads) runs while those stages are in flight.
 // app_bar completes once every thread has made its share of the fused step's
@@ -530,7 +530,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
   const bool patch = fused && p.bs == kStageTokens;
   const int32_t* r0 = p.block_tables + (size_t)lo * p.max_blocks;
 
-  // Round 1.  Lane i: member i's length and copy-on-write source.  Every lane: the
+  // First batch of loads.  Lane i: member i's length and copy-on-write source.  Every lane: the
   // block id of the warp's stage warp + W * lane, read as a prefix stage when the
   // caller's prefix reaches it (used only if the actual prefix does too).
   const int cap_pre = min(max(plen_req, 0), p.max_blocks * p.bs) / kStageTokens;
@@ -571,8 +571,8 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
 
   // This warp takes the CTA's stages warp, warp + W, ...; its stages win_base ..
   // win_base + 63 have their block ids resolved ahead, one per lane of two windows.
-  // Window 0 holds prefix ids (win0p, round 1) and own-token ids (win0t, round 2)
-  // apart, so that issuing a prefix stage never waits for a round-2 load.
+  // Window 0 holds prefix ids (win0p, first batch) and own-token ids (win0t, second batch)
+  // apart, so that issuing a prefix stage never waits for a second-batch load.
   const int first = warp, stride = W;
   const int n_w = n_all > first ? (n_all - first + stride - 1) / stride : 0;
   auto stage_id = [&](int k) -> int {  // block id of the CTA's stage k, or -1
@@ -639,7 +639,7 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     }
   };
   // The first stages that lie in the prefix: a prefix block is never one that the
-  // fused step writes.  They load after round 2 is issued, so that round 2 does not
+  // fused step writes.  They load after the second batch is issued, so that it does not
   // queue behind every warp's first stages.
   const int n_pro = n_w < C::kStages ? n_w : C::kStages;
   int n_early = 0;
@@ -647,8 +647,8 @@ __device__ __forceinline__ void group_piece(const SharedParams& s, int off_lo, i
     while (n_early < n_pro && first + stride * n_early < n_pre) issue(n_early++);
   };
 
-  // Round 2: ids of the own-token stages, the members' table check, and for a fused
-  // step each member's new-token block and the first batch of its copy reads.
+  // Second batch: ids of the own-token stages, the members' table check, and for a fused
+  // step each member's new-token block and each thread's first copy reads.
   win0t = kw >= n_pre ? stage_id(kw) : -1;
   win1 = stage_id(first + stride * (32 + lane));
   // Every member must hold the same physical blocks for the prefix: entry j of
