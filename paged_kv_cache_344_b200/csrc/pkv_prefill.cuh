@@ -588,11 +588,32 @@ __device__ __forceinline__ PpItem pp_item(const PrefillParams& p, int item) {
   return it;
 }
 
-// Orders the work items longest first (a counting sort on the number of K/V
-// tiles, one block of kSchedThreads threads), for the persistent launch, which
-// takes them in that order from an atomic counter: the longest items start
-// first and the short ones fill the tail.  Also flags bad lengths.
+// Orders the work items for the persistent launch, which takes them in that order
+// from an atomic counter.  The items of one (sequence, KV head) read the same K/V
+// tiles, so they are kept together: the units are sorted longest first (a
+// counting sort on the K/V tile count of a unit's longest item, ceil(L / 128),
+// one block of kSchedThreads threads), and each unit's items follow one another,
+// longest first.  Consecutive items start on different CTAs at about the same time
+// and stream the same tiles together, so all but the first read of a tile are L2
+// hits, while the longest units still start first and the short ones fill the
+// tail.  Also flags bad lengths.
 constexpr int kSchedThreads = 1024;  // = number of buckets
+
+// A unit's items with work (qt < n, longest at qt = n - 1) and its bucket: thread
+// order is descending cost.  n = 0 when no item of the unit has work.
+__device__ __forceinline__ void prefill_unit(const PrefillParams& p, int b, int& n, int& bucket,
+                                             bool& bad) {
+  const int Q = p.cu_q[b + 1] - p.cu_q[b];
+  const int L = p.seq_lens[b];
+  const int Lcap = min(p.max_blocks * p.bs, p.max_seq_len);
+  bad = L > Lcap || Q > L;
+  n = 0;
+  bucket = 0;
+  if (Q <= 0 || Q > min(L, Lcap)) return;  // no rows, or no consistent reading
+  n = min((Q + 2 * p.TQ - 1) / (2 * p.TQ), p.nqt);
+  const int n_kv = (min(L, Lcap) + kPpKv - 1) / kPpKv;  // the last item sees every token
+  bucket = kSchedThreads - 1 - min(n_kv, kSchedThreads - 1);
+}
 
 __global__ void __launch_bounds__(kSchedThreads)
     prefill_schedule_kernel(const PrefillParams p) {
@@ -600,17 +621,18 @@ __global__ void __launch_bounds__(kSchedThreads)
   __shared__ int warp_sum[kSchedThreads / 32];
   __shared__ int n_work;
   const int tid = threadIdx.x;
+  const int n_units = p.n_items / p.nqt;  // (sequence, KV head) pairs
   hist[tid] = 0;
   if (tid == 0) n_work = 0;
   __syncthreads();
-  // bucket kSchedThreads - 1 - min(n_kv, kSchedThreads - 1): thread order is then
-  // descending cost
-  for (int item = tid; item < p.n_items; item += kSchedThreads) {
-    const PpItem it = pp_item(p, item);
-    if (it.bad_len && it.i0 == 0 && it.kvh == 0) flag_error(PKV_DEVERR_SEQLEN);
-    if (it.n_kv > 0) {
-      atomicAdd(&hist[kSchedThreads - 1 - min(it.n_kv, kSchedThreads - 1)], 1);
-      atomicAdd(&n_work, 1);
+  for (int u = tid; u < n_units; u += kSchedThreads) {
+    int n, bucket;
+    bool bad;
+    prefill_unit(p, u / p.Hkv, n, bucket, bad);
+    if (bad && u % p.Hkv == 0) flag_error(PKV_DEVERR_SEQLEN);
+    if (n > 0) {
+      atomicAdd(&hist[bucket], n);
+      atomicAdd(&n_work, n);
     }
   }
   __syncthreads();
@@ -637,10 +659,15 @@ __global__ void __launch_bounds__(kSchedThreads)
   hist[tid] = incl - v + (tid >= 32 ? warp_sum[tid / 32 - 1] : 0);
   __syncthreads();
   int* order = p.sched + 2;
-  for (int item = tid; item < p.n_items; item += kSchedThreads) {
-    const PpItem it = pp_item(p, item);
-    if (it.n_kv > 0)
-      order[atomicAdd(&hist[kSchedThreads - 1 - min(it.n_kv, kSchedThreads - 1)], 1)] = item;
+  for (int u = tid; u < n_units; u += kSchedThreads) {
+    int n, bucket;
+    bool bad;
+    const int b = u / p.Hkv, kvh = u % p.Hkv;
+    prefill_unit(p, b, n, bucket, bad);
+    if (n > 0) {
+      int at = atomicAdd(&hist[bucket], n);
+      for (int qt = n - 1; qt >= 0; --qt) order[at++] = (b * p.nqt + qt) * p.Hkv + kvh;
+    }
   }
   if (tid == 0) {
     p.sched[0] = 0;
