@@ -1006,6 +1006,14 @@ __global__ void __launch_bounds__(kWarps * 32)
   if (!s_last) return;
   __threadfence();
   const size_t base = unit * p.max_parts * G;
+  // Each partial's weight exp2(m_q - M) / den, formed once per (partition, head)
+  // into the shared memory the stages no longer use; then every thread sums
+  // 4-float chunks of the output with kU partials' loads in flight.  (A loop over
+  // the partials one at a time was bound by L2 latency: 17-45 us per merge on the
+  // long-context workload, at the very end of the launch.)
+  constexpr int kU = 16;
+  float* s_w = reinterpret_cast<float*>(smem);  // [partition][head]
+  const bool fast = nparts * G <= kWarps * kRing / (int)sizeof(float) && D % 4 == 0;
   for (int g = warp; g < G; g += kWarps) {
     float M = -INFINITY;
     for (int q = lane; q < nparts; q += 32) M = fmaxf(M, __ldcg(&p.ws_ml[base + (size_t)q * G + g]).x);
@@ -1022,8 +1030,50 @@ __global__ void __launch_bounds__(kWarps * 32)
       s_M[g] = M;
       s_den[g] = den;
     }
+    if (fast) {
+      const float inv = 1.f / den;
+      for (int q = lane; q < nparts; q += 32)
+        s_w[q * G + g] = exp2f(__ldcg(&p.ws_ml[base + (size_t)q * G + g]).x - M) * inv;
+    }
   }
   __syncthreads();
+  if (fast) {
+    for (int c = threadIdx.x; c < G * D / 4; c += blockDim.x) {
+      const int g = c / (D / 4), d4 = c % (D / 4);
+      const float4* src = reinterpret_cast<const float4*>(p.ws_acc + (base + g) * D) + d4;
+      const size_t stride = (size_t)G * D / 4;  // float4s from one partition's row g to the next
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      int q = 0;
+      for (; q + kU <= nparts; q += kU) {
+        float4 v[kU];
+#pragma unroll
+        for (int k = 0; k < kU; ++k) v[k] = __ldcg(src + (size_t)(q + k) * stride);
+#pragma unroll
+        for (int k = 0; k < kU; ++k) {
+          const float w = s_w[(q + k) * G + g];
+          a.x = fmaf(w, v[k].x, a.x);
+          a.y = fmaf(w, v[k].y, a.y);
+          a.z = fmaf(w, v[k].z, a.z);
+          a.w = fmaf(w, v[k].w, a.w);
+        }
+      }
+      for (; q < nparts; ++q) {
+        const float4 v = __ldcg(src + (size_t)q * stride);
+        const float w = s_w[q * G + g];
+        a.x = fmaf(w, v.x, a.x);
+        a.y = fmaf(w, v.y, a.y);
+        a.z = fmaf(w, v.z, a.z);
+        a.w = fmaf(w, v.w, a.w);
+      }
+      T* o = out + g * D + 4 * d4;
+      o[0] = to_out<T>(a.x);
+      o[1] = to_out<T>(a.y);
+      o[2] = to_out<T>(a.z);
+      o[3] = to_out<T>(a.w);
+    }
+    if (threadIdx.x == 0) p.ws_count[unit] = 0u;
+    return;
+  }
   for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
     const int g = idx / D, d = idx % D;
     const float M = s_M[g];
