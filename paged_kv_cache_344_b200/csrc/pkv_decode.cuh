@@ -1015,25 +1015,37 @@ __global__ void __launch_bounds__(kWarps * 32)
   float* s_w = reinterpret_cast<float*>(smem);  // [partition][head]
   const bool fast = nparts * G <= kWarps * kRing / (int)sizeof(float) && D % 4 == 0;
   for (int g = warp; g < G; g += kWarps) {
-    float M = -INFINITY;
-    for (int q = lane; q < nparts; q += 32) M = fmaxf(M, __ldcg(&p.ws_ml[base + (size_t)q * G + g]).x);
+    float M = -INFINITY, den = 0.f;
+    if (nparts <= 32) {  // one (max, sum) a lane, read once
+      const float2 ml = lane < nparts ? __ldcg(&p.ws_ml[base + (size_t)lane * G + g])
+                                      : make_float2(-INFINITY, 0.f);
+      M = ml.x;
 #pragma unroll
-    for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-    float den = 0.f;
-    for (int q = lane; q < nparts; q += 32) {
-      const float2 ml = __ldcg(&p.ws_ml[base + (size_t)q * G + g]);
-      den += exp2f(ml.x - M) * ml.y;
+      for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+      const float e = lane < nparts ? exp2f(ml.x - M) : 0.f;
+      den = e * ml.y;
+#pragma unroll
+      for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
+      if (fast && lane < nparts) s_w[lane * G + g] = e / den;
+    } else {
+      for (int q = lane; q < nparts; q += 32) M = fmaxf(M, __ldcg(&p.ws_ml[base + (size_t)q * G + g]).x);
+#pragma unroll
+      for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+      for (int q = lane; q < nparts; q += 32) {
+        const float2 ml = __ldcg(&p.ws_ml[base + (size_t)q * G + g]);
+        den += exp2f(ml.x - M) * ml.y;
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
+      if (fast) {
+        const float inv = 1.f / den;
+        for (int q = lane; q < nparts; q += 32)
+          s_w[q * G + g] = exp2f(__ldcg(&p.ws_ml[base + (size_t)q * G + g]).x - M) * inv;
+      }
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
     if (lane == 0) {
       s_M[g] = M;
       s_den[g] = den;
-    }
-    if (fast) {
-      const float inv = 1.f / den;
-      for (int q = lane; q < nparts; q += 32)
-        s_w[q * G + g] = exp2f(__ldcg(&p.ws_ml[base + (size_t)q * G + g]).x - M) * inv;
     }
   }
   __syncthreads();
