@@ -247,9 +247,53 @@ __global__ void __launch_bounds__(kWarps * 32)
         last = __shfl_sync(kFull, last, 0);
         if (last) {
           __threadfence();
+          bool continue_after_merge = false;  // the fast merge below did the unit
           const size_t base = head_base + b + gf;
           const int nseg = gl - gf + 1;
-          for (int gg = 0; gg < G; ++gg) {
+          if (nseg <= 32 && D == 128) {
+            // Lane q holds piece q's weight exp2(m_q - M) / den of the row; then lane
+            // l sums dims 4l .. 4l + 3 over the pieces, kU pieces' loads in flight.
+            // (One piece at a time was bound by L2 latency.)
+            constexpr int kU = 8;
+            for (int gg = 0; gg < G; ++gg) {
+              const float2 ml = lane < nseg ? __ldcg(&p.ws_ml[(base + lane) * G + gg])
+                                            : make_float2(-INFINITY, 0.f);
+              float M = ml.x;
+#pragma unroll
+              for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+              const float e = lane < nseg ? exp2f(ml.x - M) : 0.f;
+              float den = e * ml.y;
+#pragma unroll
+              for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
+              const float w = e / den;
+              const float4* src = reinterpret_cast<const float4*>(p.ws_acc + (base * G + gg) * D) + lane;
+              const size_t stride = (size_t)G * D / 4;  // float4s from one piece to the next
+              float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int q0 = 0; q0 < nseg; q0 += kU) {
+                float4 v[kU];
+#pragma unroll
+                for (int k = 0; k < kU; ++k)
+                  v[k] = q0 + k < nseg ? __ldcg(src + (size_t)(q0 + k) * stride)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < kU; ++k) {
+                  const float wq = __shfl_sync(kFull, w, (q0 + k) & 31);
+                  a.x = fmaf(wq, v[k].x, a.x);
+                  a.y = fmaf(wq, v[k].y, a.y);
+                  a.z = fmaf(wq, v[k].z, a.z);
+                  a.w = fmaf(wq, v[k].w, a.w);
+                }
+              }
+              T* o = orow + gg * D + 4 * lane;
+              o[0] = to_out<T>(a.x);
+              o[1] = to_out<T>(a.y);
+              o[2] = to_out<T>(a.z);
+              o[3] = to_out<T>(a.w);
+            }
+            if (lane == 0) p.ws_count[u] = 0u;
+            continue_after_merge = true;
+          }
+          for (int gg = 0; gg < G && !continue_after_merge; ++gg) {
             float M = -INFINITY;
             for (int q = lane; q < nseg; q += 32) M = fmaxf(M, __ldcg(&p.ws_ml[(base + q) * G + gg]).x);
 #pragma unroll
@@ -270,7 +314,7 @@ __global__ void __launch_bounds__(kWarps * 32)
               orow[gg * D + d] = to_out<T>(num / den);
             }
           }
-          if (lane == 0) p.ws_count[u] = 0u;
+          if (!continue_after_merge && lane == 0) p.ws_count[u] = 0u;
         }
       }
       if (pos >= p_end) break;
