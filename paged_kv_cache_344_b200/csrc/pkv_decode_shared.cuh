@@ -300,18 +300,38 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
       __threadfence();
       const size_t base = unit * SL * G;
       auto slot_of = [&](int q) { return q < it.npp ? q : s.max_pp + (q - it.npp); };
+      // As in the decode's merge: with at most 32 pieces, lane q reads piece q's
+      // (max, sum) once and files its weight exp2(m_q - M) / den in the shared
+      // memory the stages no longer use; then each thread sums 4-float chunks of
+      // the output with kU pieces' loads in flight.
+      constexpr int kU = 8;
+      float* s_w = reinterpret_cast<float*>(smem);  // [piece][head]
+      const bool fast = tot <= 32 && tot * G * (int)sizeof(float) <= DecodeSmem<C>::kRingBytes * kWarps &&
+                        D % 4 == 0;
       for (int g = warp; g < G; g += kWarps) {
-        float M = -INFINITY;
-        for (int q = lane; q < tot; q += 32) M = fmaxf(M, __ldcg(&s.ws_ml[base + (size_t)slot_of(q) * G + g]).x);
+        float M = -INFINITY, den = 0.f;
+        if (fast) {
+          const float2 ml = lane < tot ? __ldcg(&s.ws_ml[base + (size_t)slot_of(lane) * G + g])
+                                       : make_float2(-INFINITY, 0.f);
+          M = ml.x;
 #pragma unroll
-        for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
-        float den = 0.f;
-        for (int q = lane; q < tot; q += 32) {
-          const float2 ml = __ldcg(&s.ws_ml[base + (size_t)slot_of(q) * G + g]);
-          den += exp2f(ml.x - M) * ml.y;
+          for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+          const float e = lane < tot ? exp2f(ml.x - M) : 0.f;
+          den = e * ml.y;
+#pragma unroll
+          for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
+          if (lane < tot) s_w[lane * G + g] = e / den;
+        } else {
+          for (int q = lane; q < tot; q += 32) M = fmaxf(M, __ldcg(&s.ws_ml[base + (size_t)slot_of(q) * G + g]).x);
+#pragma unroll
+          for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+          for (int q = lane; q < tot; q += 32) {
+            const float2 ml = __ldcg(&s.ws_ml[base + (size_t)slot_of(q) * G + g]);
+            den += exp2f(ml.x - M) * ml.y;
+          }
+#pragma unroll
+          for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
         }
-#pragma unroll
-        for (int off = 16; off >= 1; off /= 2) den += __shfl_xor_sync(kFull, den, off);
         if (lane == 0) {
           s_M[g] = M;
           s_den[g] = den;
@@ -319,7 +339,34 @@ __device__ __forceinline__ void shared_piece(const SharedParams& s, const Shared
       }
       __syncthreads();
       T* o = out + ((size_t)b * p.Hq + (size_t)kvh * G) * D;
-      for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+      if (fast) {
+        for (int c = threadIdx.x; c < G * D / 4; c += blockDim.x) {
+          const int g = c / (D / 4), d4 = c % (D / 4);
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q0 = 0; q0 < tot; q0 += kU) {
+            float4 v[kU];
+#pragma unroll
+            for (int k = 0; k < kU; ++k)
+              v[k] = q0 + k < tot ? __ldcg(reinterpret_cast<const float4*>(
+                                        s.ws_acc + (base + (size_t)slot_of(q0 + k) * G + g) * D) + d4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < kU; ++k) {
+              const float w = q0 + k < tot ? s_w[(q0 + k) * G + g] : 0.f;
+              a.x = fmaf(w, v[k].x, a.x);
+              a.y = fmaf(w, v[k].y, a.y);
+              a.z = fmaf(w, v[k].z, a.z);
+              a.w = fmaf(w, v[k].w, a.w);
+            }
+          }
+          T* od = o + g * D + 4 * d4;
+          od[0] = __float2bfloat16_rn(a.x);
+          od[1] = __float2bfloat16_rn(a.y);
+          od[2] = __float2bfloat16_rn(a.z);
+          od[3] = __float2bfloat16_rn(a.w);
+        }
+      }
+      for (int idx = threadIdx.x; !fast && idx < G * D; idx += blockDim.x) {
         const int g = idx / D, d = idx % D;
         float num = 0.f;
         for (int q = 0; q < tot; ++q) {
