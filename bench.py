@@ -95,6 +95,26 @@ def prime_queue():
     torch.cuda._sleep(PRIME_CYCLES)
 
 
+class L2Flush:
+    """Evicts the L2 between timed steps: a write pass over a buffer twice the L2's size,
+    then a read pass over a second one.  The write pass alone leaves the L2 full of dirty
+    lines of its buffer, and their write-back then lands inside the next timed step (about
+    3 us of a 37-52 us shared-prefix step, measured with the two orders interleaved on one
+    B200).  After the read pass the L2 holds clean lines of a buffer the step never reads."""
+
+    def __init__(self, dev_name):
+        import torch
+        n = 2 * L2_BYTES // 4
+        self.w = torch.ones(n, dtype=torch.int32, device=dev_name)
+        self.r = torch.ones(n, dtype=torch.int32, device=dev_name)
+        self.sink = torch.empty((), dtype=torch.int64, device=dev_name)
+
+    def __call__(self):
+        import torch
+        self.w.add_(1)
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
 def recorded_traffic(config: str, partition: int, kind: str = "decode"):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the current
     kernel sources (and, for decode, the same partition length); else None."""
@@ -278,7 +298,8 @@ def config_dict(args, name, wl, fused: bool, use_shared: bool, has_cow: bool, wo
                      + " (copy-on-write + cache write + decode in one launch)" if fused else
                      ("copy_blocks + " if has_cow else "") + "paged_kv_write + " + entry),
             "bytes_per_step": step_bytes,
-            "l2": (f"flushed between steps (working set {working_set / 1e9:.2f} GB)" if flush
+            "l2": (f"flushed between steps: a write pass, then a read pass, over two 0.26 GB buffers "
+                   f"(working set {working_set / 1e9:.2f} GB)" if flush
                    else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "block_size": wl.bs, "placement": "contiguous" if args.contiguous else "shuffled"}
@@ -370,7 +391,7 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
     step_bytes = cfg["bytes_per_step"]
     decode_bytes = workloads.decode_algorithmic_bytes(wl)
     flush = decode_bytes < 8 * L2_BYTES
-    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev_name) if flush else None
+    flush_l2 = L2Flush(dev_name) if flush else None
 
     def barrier():
         if world > 1:
@@ -381,9 +402,19 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
         step(d_in)
     prime_queue()  # its first launch loads the kernel; not inside a timed region
     if flush:
-        scratch.fill_(1)
-        scratch.add_(1)  # likewise the flush's kernel, which runs before every timed step
+        flush_l2()  # likewise the flush's kernels, which run before every timed step
     barrier()
+
+    # Timing events cost GPU time.  On the long-context workload a pair recorded around
+    # every fused launch added about 5 us a step, and the event just before a launch
+    # lengthened the launch it bracketed (367.4 us a step with no per-step events, 372.9 with
+    # one pair, 378.1 with two; the launch itself read 370.3 inside its pair).  So when a
+    # step is one launch and nothing runs between steps, the region holds only those
+    # launches back to back and region / K is the launch's average duration, the gaps
+    # between launches included: no per-step event is recorded.  With a flush between
+    # steps one pair brackets each fused launch; a step of several launches also gets a
+    # pair around its decode alone.
+    per_step_events = flush or not fused
 
     def timed_region():
         ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -405,16 +436,24 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
             t_start.record(stream)
             for i in range(steps):
                 if flush:
-                    scratch.add_(1)  # evict the previous step's blocks from L2 (untimed below)
-                ev_step[i][0].record(stream)
-                step(d_in, ev_dec[i])
-                ev_step[i][1].record(stream)
+                    flush_l2()  # evict the previous step's blocks from L2 (untimed below)
+                if not per_step_events:
+                    step(d_in)
+                elif fused:
+                    step(d_in, ev_dec[i])  # the step is this one launch
+                else:
+                    ev_step[i][0].record(stream)
+                    step(d_in, ev_dec[i])
+                    ev_step[i][1].record(stream)
             t_end.record(stream)
             torch.cuda.nvtx.range_pop()
             barrier()
+        region_ms = t_start.elapsed_time(t_end)
+        if not per_step_events:
+            return region_ms, [region_ms / steps] * steps, clocks
         dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
-        step_ms = [a.elapsed_time(b) for a, b in ev_step]
-        total_ms = sum(step_ms) if flush else t_start.elapsed_time(t_end)
+        step_ms = dec_ms if fused else [a.elapsed_time(b) for a, b in ev_step]
+        total_ms = sum(step_ms) if flush else region_ms
         return total_ms, dec_ms, clocks
 
     total_ms, dec_ms, clocks = timed_region()
@@ -447,6 +486,8 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
                 "kernel": kernel, "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                 "frac_of_8TBps_spec": round(achieved / SPEC_HBM_GBS, 4),
                 "decode_us": round(dec_avg_ms * 1e3, 2),
+                "launch_time": ("CUDA events around each launch" if per_step_events else
+                                "timed region / steps (launches back to back, no per-step events)"),
                 "algorithmic_bytes_per_launch": kernel_bytes,
                 "achieved_token_exact": round(workloads.decode_token_bytes(wl) / (dec_avg_ms * 1e-3) / 1e9, 1)}
     res = {"value": round(value, 1), "ms_per_step": round(ms_per_step, 5),
@@ -724,7 +765,7 @@ def run_paging(args, local_rank):
     import paged_kv_cache_344_b200 as pkv
     torch.cuda.set_device(local_rank)
     dev_name = f"cuda:{local_rank}"
-    scratch = torch.empty(2 * L2_BYTES // 4, dtype=torch.int32, device=dev_name)
+    flush_l2 = L2Flush(dev_name)
 
     def time_decode(fn, nbytes):
         flush = nbytes < 8 * L2_BYTES
@@ -736,7 +777,7 @@ def run_paging(args, local_rank):
         prime_queue()
         for a, b in ev:
             if flush:
-                scratch.add_(1)
+                flush_l2()
             a.record()
             fn()
             b.record()
