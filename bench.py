@@ -6,8 +6,10 @@ attention.  Inputs are seeded synthetic tensors resident in HBM.  The JSON line 
 
 * ``value``: algorithmic bytes of the step / step time (GB/s), summed over ranks;
 * ``tokens_per_s``: decode tokens (one per sequence) per second, summed over ranks;
-* ``roofline``: the decode kernel alone, timed with CUDA events on its stream, against the
-  measured HBM copy bandwidth;
+* ``roofline``: the decode kernel alone against the measured HBM copy bandwidth.  Its
+  launches run back to back between two CUDA events on its stream, each step on a pool of
+  inputs that the previous step did not touch, and its time is the region's over the
+  launches (a step of several launches times its decode with a pair of events instead);
 * ``e2e``: the same metric through the public API with the step's inputs copied from pinned
   host memory and the output copied back, inside the timed region;
 * ``cpu_baseline``: the fp64 oracle on this host's cores on a bounded sample (rank 0, N=1).
@@ -93,6 +95,24 @@ PRIME_CYCLES = 4_000_000  # about 2 ms at 1965 MHz
 def prime_queue():
     import torch
     torch.cuda._sleep(PRIME_CYCLES)
+
+
+MAX_POOLS = 16
+
+
+def pools_for(working_set: int) -> int:
+    """How many copies of a decode workload's inputs the timed steps cycle through.
+
+    A working set of 8 L2s or more is one pool.  A smaller one is replicated into enough
+    pools (each with its own K/V caches, q and new tokens; the block tables, lengths and
+    groups are shared, as a model's layers share them) that together they hold 8 L2s: step i
+    runs on pool i mod R, so no step finds the previous one's blocks in L2, and the launches
+    run back to back.  0: more than MAX_POOLS pools would be needed, and L2 is flushed
+    between steps instead."""
+    if working_set >= 8 * L2_BYTES:
+        return 1
+    n = -(-8 * L2_BYTES // max(working_set, 1))
+    return n if n <= MAX_POOLS else 0
 
 
 class L2Flush:
@@ -291,7 +311,7 @@ def config_dict(args, name, wl, fused: bool, use_shared: bool, has_cow: bool, wo
     step_bytes = (workloads.decode_algorithmic_bytes(wl) + workloads.write_bytes(wl) +
                   workloads.copy_bytes(wl))
     working_set = workloads.decode_algorithmic_bytes(wl)
-    flush = working_set < 8 * L2_BYTES
+    pools = pools_for(working_set)
     entry = "paged_attention_decode_shared_prefix" if use_shared else "paged_attention_decode"
     return {"workload": name, "description": DESCR.get(name, name),
             "step": (("paged_decode_step_shared_prefix" if use_shared else "paged_decode_step")
@@ -299,8 +319,10 @@ def config_dict(args, name, wl, fused: bool, use_shared: bool, has_cow: bool, wo
                      ("copy_blocks + " if has_cow else "") + "paged_kv_write + " + entry),
             "bytes_per_step": step_bytes,
             "l2": (f"flushed between steps: a write pass, then a read pass, over two 0.26 GB buffers "
-                   f"(working set {working_set / 1e9:.2f} GB)" if flush
-                   else f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)"),
+                   f"(working set {working_set / 1e9:.2f} GB)" if pools == 0 else
+                   f"inputs larger than L2 ({working_set / 1e9:.2f} GB vs 0.13 GB L2)" if pools == 1
+                   else f"inputs larger than L2: {pools} pools of {working_set / 1e9:.2f} GB (own K/V, "
+                        f"q and new tokens; shared tables), step i on pool i mod {pools}"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
             "block_size": wl.bs, "placement": "contiguous" if args.contiguous else "shuffled"}
 
@@ -390,16 +412,22 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
     cfg = config_dict(args, name, wl, fused, use_shared, has_cow, world)
     step_bytes = cfg["bytes_per_step"]
     decode_bytes = workloads.decode_algorithmic_bytes(wl)
-    flush = decode_bytes < 8 * L2_BYTES
+    n_pools = pools_for(decode_bytes)
+    flush = n_pools == 0
     flush_l2 = L2Flush(dev_name) if flush else None
+    d_ins = [d_in]
+    for r in range(1, n_pools):
+        d_r = workloads.device_tensors(wl, dev_name, seed_offset=rank + 1000 * r)
+        d_r.update(meta)
+        d_ins.append(d_r)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(warmup):
-        step(d_in)
+    for i in range(max(warmup, len(d_ins))):  # every pool at least once
+        step(d_ins[i % len(d_ins)])
     prime_queue()  # its first launch loads the kernel; not inside a timed region
     if flush:
         flush_l2()  # likewise the flush's kernels, which run before every timed step
@@ -437,13 +465,14 @@ def run_decode(args, name, rank, world, local_rank, steps, warmup, with_e2e, wit
             for i in range(steps):
                 if flush:
                     flush_l2()  # evict the previous step's blocks from L2 (untimed below)
+                d_i = d_ins[i % len(d_ins)]
                 if not per_step_events:
-                    step(d_in)
+                    step(d_i)
                 elif fused:
-                    step(d_in, ev_dec[i])  # the step is this one launch
+                    step(d_i, ev_dec[i])  # the step is this one launch
                 else:
                     ev_step[i][0].record(stream)
-                    step(d_in, ev_dec[i])
+                    step(d_i, ev_dec[i])
                     ev_step[i][1].record(stream)
             t_end.record(stream)
             torch.cuda.nvtx.range_pop()

@@ -61,3 +61,16 @@ def test_both_arms_report_the_same_config():
         assert a["workload"] == name and a["block_size"] == wl.bs
         assert a["bytes_per_step"] == (workloads.decode_algorithmic_bytes(wl) +
                                        workloads.write_bytes(wl) + workloads.copy_bytes(wl))
+
+
+def test_pools_hold_eight_l2s_or_flush():
+    """Small working sets are cycled through enough pools to hold 8 L2s; beyond
+    MAX_POOLS pools the bench flushes L2 instead."""
+    L2 = bench.L2_BYTES
+    assert bench.pools_for(8 * L2) == 1 and bench.pools_for(20 * L2) == 1
+    for ws in (158_371_328, 211_064_720, L2, 8 * L2 - 1):
+        n = bench.pools_for(ws)
+        assert n >= 2 and n * ws >= 8 * L2 and (n - 1) * ws < 8 * L2
+    assert bench.pools_for(8 * L2 // bench.MAX_POOLS) == bench.MAX_POOLS
+    assert bench.pools_for(8 * L2 // bench.MAX_POOLS - 1) == 0
+    assert bench.pools_for(4096) == 0
