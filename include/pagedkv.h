@@ -25,7 +25,11 @@
  *     pointer after the call returns.  Apart from the decode workspace, which
  *     the caller provides, it allocates no device memory.
  *   - Streams: every call enqueues its work on `stream` (NULL = the legacy
- *     default stream) and returns without synchronising.
+ *     default stream) and returns without synchronising.  Kernels are
+ *     launched with programmatic stream serialization: a launch's CTAs may be
+ *     placed while the kernel before it in the stream finishes, but each waits
+ *     for that kernel to complete before it reads or writes global memory, so
+ *     every access keeps the stream order.
  *   - Alignment: every data pointer must be 16-byte aligned.
  *   - Errors: a call returns PKV_OK or a negative status.  It validates
  *     arguments on the host before enqueueing anything, and on a validation

@@ -10,6 +10,7 @@
 #include <atomic>
 #include <cmath>
 #include <mutex>
+#include <utility>
 
 #include "pkv_decode_balanced.cuh"
 #include "pkv_decode_shared.cuh"
@@ -122,6 +123,29 @@ int make_stage_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t r
   return PKV_OK;
 }
 
+// Launches a kernel with programmatic stream serialization: its CTAs may be placed
+// while the kernel before it in the stream finishes (once that kernel's CTAs have
+// all begun), and each waits in launch_overlap_entry() for that kernel to complete
+// before it touches global memory.  Back-to-back steps thus overlap one grid's
+// launch and CTA set-up with the previous grid's last CTAs.  Returns the launch's
+// error, else any earlier asynchronous one.
+template <typename... Params, typename... Args>
+cudaError_t launch_overlapped(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // Raises the dynamic shared-memory limit of a kernel once per device.  `done`
 // must be distinct for every kernel (all decode kernels share one C++ type).
 template <typename Kernel>
@@ -222,8 +246,7 @@ int launch_decode(const pkv::DecodeParams& p, int B, const CUtensorMap& mk, cons
   int rc = ensure_smem(kernel, smem, smem_set);
   if (rc != PKV_OK) return rc;
   dim3 grid((unsigned)p.Hkv, (unsigned)p.max_parts, (unsigned)B);
-  kernel<<<grid, pkv::kWarps * 32, smem, stream>>>(p, mk, mv);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_overlapped(kernel, grid, dim3(pkv::kWarps * 32), smem, stream, p, mk, mv);
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
@@ -253,8 +276,8 @@ int launch_balanced(const pkv::DecodeParams& p, const CUtensorMap& mk, const CUt
   }
   const int forced = g_decode_ctas.load(std::memory_order_relaxed);
   if (forced > 0) ctas = std::min(forced, pkv::kBalancedMaxCtas);
-  kernel<<<ctas, pkv::kWarps * 32, pkv::BalancedSmem<C>::bytes(p.B), stream>>>(p, mk, mv);
-  e = cudaGetLastError();
+  e = launch_overlapped(kernel, dim3(ctas), dim3(pkv::kWarps * 32), pkv::BalancedSmem<C>::bytes(p.B),
+                        stream, p, mk, mv);
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
@@ -345,8 +368,8 @@ int launch_shared(const pkv::SharedParams& sp, int64_t items, const CUtensorMap&
   static std::atomic<uint64_t> smem_set{0};
   int rc = ensure_smem(kernel, smem, smem_set);
   if (rc != PKV_OK) return rc;
-  kernel<<<(unsigned)items, pkv::kWarps * 32, smem, stream>>>(sp, mk, mv);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_overlapped(kernel, dim3((unsigned)items), dim3(pkv::kWarps * 32), smem,
+                                    stream, sp, mk, mv);
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
@@ -373,8 +396,8 @@ int launch_group(const pkv::SharedParams& sp, int64_t items, const CUtensorMap& 
   static std::atomic<uint64_t> smem_set{0};
   int rc = ensure_smem(kernel, smem, smem_set);
   if (rc != PKV_OK) return rc;
-  kernel<<<(unsigned)items, W * 32, smem, stream>>>(sp, mk, mv);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_overlapped(kernel, dim3((unsigned)items), dim3(W * 32), smem, stream, sp,
+                                    mk, mv);
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
@@ -401,10 +424,10 @@ int paged_kv_write(const void* k, const void* v, void* k_cache, void* v_cache,
   const int threads = 256;
   const int64_t gy = std::min<int64_t>(std::max<int64_t>(ceil_div(row_vec, threads), 1), 65535);
   dim3 grid((unsigned)N, (unsigned)gy);
-  pkv::kv_write_kernel<<<grid, threads, 0, stream>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), slot_mapping, row_vec, num_blocks * block_size);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_overlapped(
+      pkv::kv_write_kernel, grid, dim3(threads), 0, stream, static_cast<const uint4*>(k),
+      static_cast<const uint4*>(v), static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+      slot_mapping, row_vec, num_blocks * block_size);
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 
@@ -842,8 +865,7 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
   auto launch = [&](auto kernel, size_t smem, std::atomic<uint64_t>& set, int threads) -> int {
     int rc2 = ensure_smem(kernel, smem, set);
     if (rc2 != PKV_OK) return rc2;
-    kernel<<<grid, threads, smem, stream>>>(p, mq, mk, mv);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_overlapped(kernel, grid, dim3(threads), smem, stream, p, mq, mk, mv);
     return e == cudaSuccess ? PKV_OK : cuda_fail(e);
   };
   static std::atomic<uint64_t> pp64{0}, pp128{0}, set64{0}, set128{0}, set256{0};
@@ -852,8 +874,8 @@ int paged_attention_prefill(void* out, const void* q, const void* k_cache, const
     // per SM takes them in that order.  Without: one CTA per item.
     if (workspace) {
       p.sched = static_cast<int*>(workspace);
-      pkv::prefill_schedule_kernel<<<1, pkv::kSchedThreads, 0, stream>>>(p);
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launch_overlapped(pkv::prefill_schedule_kernel, dim3(1),
+                                        dim3(pkv::kSchedThreads), 0, stream, p);
       if (e != cudaSuccess) return cuda_fail(e);
       int sms = 0;
       if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e);
@@ -884,10 +906,9 @@ int copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping, int6
   const int threads = 256;
   const int64_t gy = std::min<int64_t>(std::max<int64_t>(ceil_div(block_vec, threads * 4), 1), 65535);
   dim3 grid((unsigned)P, (unsigned)gy);
-  pkv::copy_blocks_kernel<<<grid, threads, 0, stream>>>(static_cast<uint4*>(k_cache),
-                                                        static_cast<uint4*>(v_cache),
-                                                        block_mapping, block_vec, num_blocks);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_overlapped(pkv::copy_blocks_kernel, grid, dim3(threads), 0, stream,
+                                    static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                                    block_mapping, block_vec, num_blocks);
   return e == cudaSuccess ? PKV_OK : cuda_fail(e);
 }
 

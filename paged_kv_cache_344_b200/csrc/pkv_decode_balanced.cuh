@@ -56,6 +56,7 @@ template <class C, typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32)
     paged_decode_balanced_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                                  const __grid_constant__ CUtensorMap tmV) {
+  launch_overlap_entry();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

@@ -833,6 +833,7 @@ template <class C, int D, int W>
 __global__ void __launch_bounds__(W * 32, D <= 128 ? 2 : 1)
     paged_decode_group_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
                               const __grid_constant__ CUtensorMap tmV) {
+  launch_overlap_entry();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -860,6 +861,7 @@ template <class C2, class C1, int D>
 __global__ void __launch_bounds__(kWarps * 32)
     paged_decode_shared_kernel(const SharedParams s, const __grid_constant__ CUtensorMap tmK,
                                const __grid_constant__ CUtensorMap tmV) {
+  launch_overlap_entry();
   static_assert(DecodeSmem<C2>::kBytes == DecodeSmem<C1>::kBytes, "consumers share the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

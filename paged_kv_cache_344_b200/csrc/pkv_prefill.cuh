@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     paged_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                          const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV) {
+  launch_overlap_entry();
   using S = PrefillSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -617,6 +618,7 @@ __device__ __forceinline__ void prefill_unit(const PrefillParams& p, int b, int&
 
 __global__ void __launch_bounds__(kSchedThreads)
     prefill_schedule_kernel(const PrefillParams p) {
+  launch_overlap_entry();
   __shared__ int hist[kSchedThreads];
   __shared__ int warp_sum[kSchedThreads / 32];
   __shared__ int n_work;
@@ -686,6 +688,7 @@ __global__ void __launch_bounds__(kPpThreads, 1)
     paged_prefill_pp_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmK,
                             const __grid_constant__ CUtensorMap tmV) {
+  launch_overlap_entry();
   using S = PpSmem<D>;
   constexpr int R = S::kRing;
   constexpr int kBoxes = kPpKv / kStageTokens;  // 16-token boxes per K/V tile

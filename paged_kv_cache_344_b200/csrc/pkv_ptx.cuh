@@ -23,6 +23,21 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialization and opens with launch_overlap_entry(): it lets
+// the next such launch in the stream place its CTAs as this grid's CTAs retire
+// (griddepcontrol.launch_dependents; the next grid starts only once every CTA of
+// this one has begun or exited), then waits until the kernel before it in the
+// stream has completed and its memory is visible (griddepcontrol.wait).  Nothing
+// before that wait touches global memory, so the order of every input, output and
+// workspace access is the stream order.  What overlaps is the next grid's launch
+// and CTA set-up with this grid's last CTAs.  Without the launch attribute both
+// instructions do nothing.
+__device__ __forceinline__ void launch_overlap_entry() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                : "memory");

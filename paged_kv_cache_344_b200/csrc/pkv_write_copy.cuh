@@ -16,6 +16,7 @@ __global__ void __launch_bounds__(256)
     kv_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                     uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                     const int64_t* __restrict__ slot_mapping, int64_t row_vec, int64_t num_slots) {
+  launch_overlap_entry();
   const int64_t n = blockIdx.x;
   const int64_t s = slot_mapping[n];
   if (s < 0) return;
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(256)
     copy_blocks_kernel(uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
                        const int64_t* __restrict__ block_mapping, int64_t block_vec,
                        int64_t num_blocks) {
+  launch_overlap_entry();
   const int64_t i = blockIdx.x;
   const int64_t src = block_mapping[2 * i];
   const int64_t dst = block_mapping[2 * i + 1];
