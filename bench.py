@@ -596,7 +596,9 @@ def run_e2e(step, d_in, out, has_cow, stream, step_bytes, wl, world, dev_name, s
     e0.record(stream)  # created now, not inside the region
     e1.record(stream)
     barrier()
-    e2e_steps = max(10, steps // 4)
+    e2e_steps = max(10, steps)
+    with torch.cuda.stream(copy_s):
+        prime_queue()  # the host queues the first steps while the copy stream waits
     e0.record(copy_s)
     e2e_run(e2e_steps)
     e1.record(copy_s)
