@@ -426,6 +426,16 @@ enum { PKV_PATH_AUTO = 0, PKV_PATH_CUDA_CORES = 1, PKV_PATH_TENSOR_CORES = 2 };
 int pkv_set_decode_path(int mode);
 
 /*
+ * Launch overlap, set for the whole process: 1 (default) launches every kernel
+ * with programmatic stream serialization (a launch's CTAs may be placed while the
+ * kernel before it in the stream finishes; each waits for that kernel before it
+ * touches global memory); 0 launches them in plain stream order, each grid
+ * starting once the previous kernel has completed.  Results are the same bits
+ * either way.  Returns the previous setting, or PKV_ERR_INVALID_ARG.
+ */
+int pkv_set_launch_overlap(int enabled);
+
+/*
  * Kernel used by paged_attention_prefill, set for the whole process (for
  * testing and measuring both):
  *   PKV_PREFILL_AUTO         D <= 128: the warp-specialised kernel with two

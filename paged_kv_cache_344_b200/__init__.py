@@ -115,6 +115,8 @@ def lib() -> ctypes.CDLL:
     L.pkv_set_prefill_path.restype = i32
     L.pkv_set_decode_path.argtypes = [i32]
     L.pkv_set_decode_path.restype = i32
+    L.pkv_set_launch_overlap.argtypes = [i32]
+    L.pkv_set_launch_overlap.restype = i32
     L.pkv_debug_stalled_wait.argtypes = [ctypes.c_void_p]
     L.pkv_debug_stalled_wait.restype = i32
     L.pkv_set_decode_split.argtypes = [i32]
@@ -329,6 +331,14 @@ def set_decode_path(mode: int) -> int:
     r = lib().pkv_set_decode_path(int(mode))
     _check("pkv_set_decode_path", min(r, 0))
     return r
+
+
+def set_launch_overlap(enabled: bool) -> bool:
+    """Launch kernels with programmatic stream serialization (default) or in plain
+    stream order, process-wide; returns the old setting."""
+    r = lib().pkv_set_launch_overlap(1 if enabled else 0)
+    _check("pkv_set_launch_overlap", min(r, 0))
+    return bool(r)
 
 
 def set_prefill_path(mode: int) -> int:

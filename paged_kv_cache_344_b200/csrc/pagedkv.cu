@@ -129,6 +129,8 @@ int make_stage_map(CUtensorMap* map, const void* base, int D, int Hkv, int64_t r
 // before it touches global memory.  Back-to-back steps thus overlap one grid's
 // launch and CTA set-up with the previous grid's last CTAs.  Returns the launch's
 // error, else any earlier asynchronous one.
+std::atomic<int> g_launch_overlap{1};  // pkv_set_launch_overlap
+
 template <typename... Params, typename... Args>
 cudaError_t launch_overlapped(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args&&... args) {
@@ -141,7 +143,7 @@ cudaError_t launch_overlapped(void (*kernel)(Params...), dim3 grid, dim3 block, 
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = g_launch_overlap.load(std::memory_order_relaxed) ? 1 : 0;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -1029,6 +1031,11 @@ int pkv_debug_stalled_wait(pkv_stream_t stream_) {
 int pkv_set_prefill_path(int mode) {
   if (mode != PKV_PREFILL_AUTO && mode != PKV_PREFILL_SINGLE_TILE) return PKV_ERR_INVALID_ARG;
   return g_prefill_path.exchange(mode);
+}
+
+int pkv_set_launch_overlap(int enabled) {
+  if (enabled != 0 && enabled != 1) return PKV_ERR_INVALID_ARG;
+  return g_launch_overlap.exchange(enabled);
 }
 
 int pkv_set_decode_path(int mode) {

@@ -160,6 +160,13 @@ def test_decode_cta_selector(lib):
         pkv.set_decode_ctas(-1)
 
 
+def test_launch_overlap_switch(lib):
+    old = pkv.set_launch_overlap(False)
+    assert pkv.set_launch_overlap(True) is False
+    assert pkv.set_launch_overlap(old) is True
+    assert lib.pkv_set_launch_overlap(2) == ERR_ARG
+
+
 def test_decode_path_selector(lib):
     old = pkv.set_decode_path(pkv.PKV_PATH_TENSOR_CORES)
     assert pkv.set_decode_path(pkv.PKV_PATH_CUDA_CORES) == pkv.PKV_PATH_TENSOR_CORES

@@ -116,3 +116,35 @@ def test_back_to_back_group_steps():
         assert_attention_close(widen(o), ref, wl.dtype, f"group step {t}")
     assert to_host_bits(kcache).tobytes() == kc.tobytes()
     assert to_host_bits(vcache).tobytes() == vc.tobytes()
+
+
+def test_launch_overlap_off_gives_the_same_bits():
+    """With the launch overlap switched off the kernels start in plain stream order:
+    the same steps give the same bits."""
+    lens = [5, 130, 2050, 4100, 7, 1000]
+    wl = workloads.custom("steps_off", "bf16", len(lens), 32, 8, 128, 16, lens, seed=65)
+    host = workloads.host_tensors(wl)
+    steps = _steps(wl)
+    bt = torch.from_numpy(wl.block_tables).cuda()
+    msl = wl.max_seq_len + T
+    n = pkv.paged_attention_decode_workspace_size(wl.B, wl.Hq, wl.Hkv, wl.D, msl, wl.bs, 0)
+    results = []
+    for overlap in (True, False):
+        old = pkv.set_launch_overlap(overlap)
+        try:
+            kcache = to_device(host["k_cache"], wl.dtype)
+            vcache = to_device(host["v_cache"], wl.dtype)
+            ws = torch.zeros(max(n, 1), dtype=torch.uint8, device="cuda")
+            outs = []
+            for q, kn, vn, sl in _device_steps(wl, steps):
+                o = torch.empty_like(q)
+                pkv.paged_decode_step(o, q, kn, vn, kcache, vcache, bt, sl, msl, wl.scale,
+                                      workspace=ws)
+                outs.append(o)
+            torch.cuda.synchronize()
+            results.append(([to_host_bits(o).tobytes() for o in outs],
+                            to_host_bits(kcache).tobytes(), to_host_bits(vcache).tobytes()))
+        finally:
+            pkv.set_launch_overlap(old)
+    assert results[0] == results[1]
+    assert pkv.device_errors() == 0
